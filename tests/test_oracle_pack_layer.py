@@ -1,0 +1,48 @@
+"""Pins for the packed layout and the whole-layer invariants of the oracle."""
+import numpy as np
+
+from oracle import slim_oracle as O
+from post_weight_quantization_hessian_b200 import synthetic as syn
+
+
+def test_pack_hand_example():
+    # two groups of 32 at bits [1, 3], average 2 -> 64 * 2 / 32 = 4 words per row
+    codes = np.zeros((1, 64), dtype=np.int64)
+    codes[0, :32] = 1                 # stream bits 0..31 all set -> word 0 = 0xFFFFFFFF
+    codes[0, 32] = 5                  # stream bits 32..34 = 1,0,1 -> word 1 bits 0..2 = 0b101
+    codes[0, 42] = 7                  # stream bits 62,63,64 -> word 1 bits 30,31 and word 2 bit 0
+    words = O.pack_codes(codes, [1, 3], 32, 2)
+    assert words.tolist() == [[0xFFFFFFFF, 0xC0000005, 0x1, 0x0]]
+    assert np.array_equal(O.unpack_codes(words, [1, 3], 32, 64), codes)
+
+
+def test_pack_roundtrip_and_fast_path():
+    rng = np.random.default_rng(0)
+    bits = [3, 1, 2, 2, 1, 3]
+    g = 32
+    codes = np.concatenate([rng.integers(0, 2 ** b, size=(5, g)) for b in bits], axis=1)
+    w1 = O.pack_codes(codes, bits, g, 2)
+    assert w1.shape == (5, 6 * 32 * 2 // 32)
+    assert np.array_equal(O.pack_codes_fast(codes, bits, g, 2), w1)
+    assert np.array_equal(O.unpack_codes(w1, bits, g, 6 * g), codes)
+
+
+def test_tiny_layer_invariants():
+    spec = syn.TINY
+    W = syn.make_weight(spec)
+    X = syn.activations_f64(spec)
+    r = O.quantize_layer(W, X, spec.group, spec.avg_bits, spec.lam, spec.n_tau, final_kl=True)
+    k = spec.k
+    assert sorted(r.order.tolist()) == list(range(k))
+    assert r.sba.bits.sum() == k * spec.avg_bits
+    assert (r.sba.bits == 3).sum() == (r.sba.bits == 1).sum() == r.sba.p_star
+    assert np.all(r.h > 0)
+    # every dequantized value sits on its group's grid
+    for c, b in enumerate(r.sba.bits):
+        q = r.sqc.codes[:, c * spec.group:(c + 1) * spec.group]
+        assert q.min() >= 0 and q.max() <= 2 ** b - 1
+    assert np.array_equal(O.unpack_codes(r.words, r.sba.bits, spec.group, spec.n), r.sqc.codes)
+    # the seeded salient columns' groups outrank the rest
+    sal = syn.salient_columns(spec) // spec.group
+    assert set(r.order[:1].tolist()) <= set(sal.tolist())
+    assert r.kl_final is not None and r.kl_final >= 0
