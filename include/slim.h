@@ -1,0 +1,213 @@
+/*
+ * slim.h - C ABI of libslim, a B200 (sm_100a) implementation of the per-layer
+ * quantize path of SliM-LLM (salience-driven group-wise mixed-precision
+ * post-training quantization of LLM weights).
+ *
+ * Sources that define the operations (web pages about the method):
+ *   [P1] rkmt.cn, "【ICML 2025】SliM-LLM 论文解读", sections 核心设计
+ *        (组件一 SBA, 组件二 SQC), 实验设计与结果 (评测协议), FAQ.
+ *   [P2] atlas.scime.ai summary of the SliM-LLM paper, section Approach.
+ *   [P3] briefgpt.xyz, arXiv 2405.14917 abstract.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - W is the layer weight, float32, m x n, row-major (out x in, the layout of
+ *   a PyTorch Linear). X is the calibration activations, N x n, row-major,
+ *   float32 (SLIM_X_F32) or bf16 bit patterns (SLIM_X_BF16).
+ * - Columns are split into k = n / group consecutive groups; group is 32, 64
+ *   or 128 and must divide n. avg_bits is the average bit-width b (2..7); the
+ *   groups get b-1, b or b+1 bits.
+ * - Every array argument is DEVICE memory owned by the caller unless marked
+ *   HOST. The library keeps no state between calls and never frees caller
+ *   memory. Arrays must not overlap. W must be 16-byte aligned and X too.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Work is ordered on it. Each call enqueues its kernels, then waits for the
+ *   stream to drain and reads the call's device status word, so that it can
+ *   return device-side failures (SLIM_ENOTPD, SLIM_ETIMEOUT). Outputs are
+ *   complete when the call returns SLIM_OK.
+ * - Workspace: `ws` is device scratch of at least the size the matching
+ *   *_workspace_bytes function returns, 256-byte aligned. ws == NULL makes the
+ *   call allocate (cudaMallocAsync on `stream`) and free it itself.
+ * - Errors are returned, never raised: on any status other than SLIM_OK the
+ *   outputs are unspecified. Arguments are validated before any launch.
+ * - Calls on the same device that share a workspace must not overlap.
+ */
+#ifndef SLIM_H
+#define SLIM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SLIM_OK = 0,
+  SLIM_EINVAL = 1,    /* bad argument (size, group, bits, NULL pointer, alignment) */
+  SLIM_ENOMEM = 2,    /* the library could not allocate device memory */
+  SLIM_ECUDA = 3,     /* a CUDA runtime call failed; see slim_last_cuda_error() */
+  SLIM_ETIMEOUT = 4,  /* a device-side wait ran past its limit; the kernel stopped */
+  SLIM_ENOTPD = 5,    /* the damped Hessian has no Cholesky factor */
+  SLIM_ENODEV = 6,    /* no sm_100 device is current */
+  SLIM_EINJECTED = 7, /* a failure was injected on the host (SLIM_FAULT=<stage>) */
+  SLIM_ERANGE = 8     /* an input does not fit the fp16 tensor-core operands of the
+                         SBA scoring (|x| or 256 |w| above 65504) */
+} slim_status;
+
+typedef enum { SLIM_X_F32 = 0, SLIM_X_BF16 = 1 } slim_xdtype;
+
+/* Human-readable text of a status code. Never NULL. */
+const char* slim_status_string(int status);
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+const char* slim_last_cuda_error(void);
+/* Library version string. */
+const char* slim_version(void);
+
+/* Number of SBA candidates, floor(k / 2) + 1 ([P1] 组件一 SBA: the search
+ * range of the promoted-group count p is [0, k/2]). */
+int slim_num_candidates(int64_t n, int group);
+
+/* Packed-code words per row: n * avg_bits / 32. */
+int64_t slim_row_words(int64_t n, int avg_bits);
+
+/* Number of CUDA kernels this library has launched in this process so far
+ * (all threads, all calls). Differences around a call count its launches. */
+int64_t slim_launch_count(void);
+
+/* ------------------------------------------------------------------------
+ * slim_hessian: H = 2 X^T X ([P1] 组件一 SBA: the Hessian is approximated
+ * from calibration activations, no backpropagation).
+ *   X   device, N x n, row-major, dtype xdtype.
+ *   H   device, n x n float64, row-major; both triangles are written.
+ * bf16 X runs on the tensor cores (tcgen05, fp32 accumulation over token
+ * slices, fp64 sum of the slices); float32 X runs an fp64-accumulating
+ * CUDA-core kernel. Requires n % 32 == 0 and N >= 1.
+ */
+size_t slim_hessian_workspace_bytes(int64_t N, int64_t n, int xdtype);
+int slim_hessian(const void* X, int xdtype, int64_t N, int64_t n, double* H,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * slim_hinv_diag: h_j = [H_d^-1]_jj, the inverse-Hessian diagonal used by the
+ * salience formula ([P1] 组件一 SBA, delta formula).
+ *   H_d = H with every zero diagonal entry set to 1, plus
+ *         alpha * mean(diag) on the diagonal (alpha = 0.01 is the usual damping).
+ *   H   device, n x n float64 row-major, read only (symmetric; the lower
+ *       triangle is used).
+ *   h   device, n float64.
+ * Blocked fp64 Cholesky H_d = L L^T, blocked inverse of L, then column sums
+ * of squares of L^-1. Returns SLIM_ENOTPD if a pivot is not positive.
+ */
+size_t slim_hinv_diag_workspace_bytes(int64_t n);
+int slim_hinv_diag(const double* H, int64_t n, double alpha, double* h,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * slim_salience: delta_ij = w_ij^2 / h_j^2 ([P1] 组件一 SBA), group means
+ * S_c = mean over rows and the group's columns ([P2] Approach: allocation by
+ * average group salience), and the groups in descending S (equal values: the
+ * lower group index first).
+ *   W      device m x n float32;  h device n float64.
+ *   S      device k float64;      order device k int32.
+ */
+size_t slim_salience_workspace_bytes(int64_t m, int64_t n, int group);
+int slim_salience(const float* W, int64_t m, int64_t n, const double* h, int group,
+                  double* S, int32_t* order, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * slim_sba_search: salience-determined bit allocation ([P1] 组件一 SBA,
+ * [P2] Approach). For p = 0 .. floor(k/2): groups order[0..p) get avg_bits+1,
+ * groups order[k-p..k) get avg_bits-1, the rest avg_bits (balanced counts, so
+ * the average stays avg_bits). Each candidate is scored by
+ *   KL_p = mean over the N tokens of KL(softmax(x W^T) || softmax(x W_p^T)),
+ * softmax over the m output features, W_p the per-group min-max round-to-
+ * nearest dequantization of W under that allocation. p* is the smallest p
+ * with the least KL.
+ *   order    device k int32 (from slim_salience).
+ *   kl       device P float64 (P = slim_num_candidates), may be NULL.
+ *   p_star   device int32, may be NULL.
+ *   bits     device k uint8 (the allocation at p*).
+ * All candidates are scored in one pass over X: a tensor-core kernel keeps,
+ * per token tile, the outputs X W^T and the quantization-error outputs in
+ * tensor memory, and updates them group pair by group pair as p grows. The
+ * tensor-core operands are fp16 (X converted exactly from bf16; the weight
+ * arrays scaled by 2^8): inputs with |x| > 65504 or |w| > 255 return
+ * SLIM_ERANGE.
+ */
+size_t slim_sba_workspace_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group);
+int slim_sba_search(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N,
+                    int group, int avg_bits, const int32_t* order, double* kl, int32_t* p_star,
+                    uint8_t* bits, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * slim_sqc: salience-weighted quantizer calibration ([P1] 组件二 SQC,
+ * [P2] Approach, [P3]). For each (row i, group c) with b = bits[c]:
+ *   mask   w < mu - 3 sigma or w > mu + 3 sigma (population sigma);
+ *   s0, z0 min-max scale (hi - lo)/(2^b - 1) and float zero -lo/s0;
+ *   tau_t  = (1 - lambda) + 2 lambda t / (n_tau - 1), t < n_tau (tau = 1 if n_tau = 1);
+ *   q      = clamp(rint(w / (tau_t s0) + z0), 0, 2^b - 1), w_hat = tau_t s0 (q - z0);
+ *   E_t    = mean_{mask} delta e^2 + mean_{not mask} delta e^2, e = w - w_hat,
+ *            delta = w^2 / h_j^2;
+ *   t*     = the smallest t with the least E_t (all arithmetic in fp64).
+ * Outputs:
+ *   codes    device uint32, m x slim_row_words(n, avg_bits): row i is a
+ *            little-endian bit stream; group c's g codes (bits[c] bits each,
+ *            column order, least significant bit first) follow the groups
+ *            before it. sum(bits) must equal k * avg_bits.
+ *   scale, zero  device m x k float32 (w_hat = scale * (q - zero)).
+ *   tau_idx  device m x k uint8 (t*), may be NULL.
+ * A group whose values are all equal stores scale 1, zero -lo, codes 0, t* 0.
+ * Requires n_tau in [1, 256], 0 <= lambda < 1. lambda is taken as given
+ * (double), so the tau grid is the exact fp64 expression above.
+ */
+int slim_sqc(const float* W, int64_t m, int64_t n, const double* h, const uint8_t* bits,
+             int group, int avg_bits, double lambda, int n_tau, uint32_t* codes, float* scale,
+             float* zero, uint8_t* tau_idx, void* stream);
+
+/* ------------------------------------------------------------------------
+ * slim_quantize_layer: the whole path, hessian -> hinv_diag -> salience ->
+ * sba_search -> sqc ([P1] 核心设计: SBA allocates bits between groups, SQC
+ * calibrates each group's quantizer), with damping alpha = 0.01.
+ *   codes, scale, zero: as slim_sqc.  bits: device k uint8.
+ */
+size_t slim_workspace_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group, int avg_bits);
+int slim_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N,
+                        int group, int avg_bits, double lambda, int n_tau, uint32_t* codes,
+                        float* scale, float* zero, uint8_t* bits, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/* Optional diagnostics of slim_quantize_layer_ex. Pointers may be NULL. */
+typedef struct {
+  double* H;          /* device n x n float64 */
+  double* h;          /* device n float64 */
+  double* S;          /* device k float64 */
+  int32_t* order;     /* device k int32 */
+  double* kl;         /* device P float64 */
+  uint8_t* tau_idx;   /* device m x k uint8 */
+  int32_t p_star;     /* HOST, written by the call */
+  float stage_ms[8];  /* HOST, written: stages hessian, hinv_diag, salience, sba_search, sqc,
+                         total, then the tensor-core kernels alone: hessian (bf16 X), sba scoring */
+} slim_diag;
+
+int slim_quantize_layer_ex(const float* W, int64_t m, int64_t n, const void* X, int xdtype,
+                           int64_t N, int group, int avg_bits, double lambda, int n_tau,
+                           uint32_t* codes, float* scale, float* zero, uint8_t* bits, void* ws,
+                           size_t ws_bytes, void* stream, slim_diag* diag);
+
+/* ------------------------------------------------------------------------
+ * slim_quantize_layer_host: slim_quantize_layer on HOST arrays (W, X in;
+ * codes, scale, zero, bits out; same layouts). The call allocates device
+ * buffers, copies inputs to the device, runs the path, copies results back
+ * and frees. Pinned host memory makes the copies asynchronous-capable and
+ * fast; pageable memory works too.
+ */
+int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X, int xdtype,
+                             int64_t N, int group, int avg_bits, double lambda, int n_tau,
+                             uint32_t* codes, float* scale, float* zero, uint8_t* bits,
+                             void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SLIM_H */

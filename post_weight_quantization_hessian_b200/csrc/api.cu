@@ -1,0 +1,421 @@
+// libslim C ABI: argument validation, workspace carving, stage sequencing on
+// the caller's stream, device status mapping and per-stage timing.
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <atomic>
+
+#include "common.cuh"
+#include "../../include/slim.h"
+
+namespace slim {
+// stage launchers (defined in the kernel files)
+cudaError_t launch_hessian(const void* X, int xdtype, int64_t N, int64_t n, double* H, void* part, DevStatus* st,
+                           int num_sms, cudaStream_t s, cudaEvent_t* kev);
+size_t hessian_ws_bytes(int64_t N, int64_t n, int xdtype);
+size_t hinv_workspace_doubles(int64_t n);
+cudaError_t launch_hinv(const double* H, int64_t n, double alpha, double* h, double* ws, DevStatus* st,
+                        cudaStream_t s);
+int salience_row_blocks(int64_t m);
+cudaError_t launch_salience(const float* W, int64_t m, int64_t n, const double* h, int group, double* S,
+                            int32_t* order, double* part, cudaStream_t st);
+size_t sba_ws_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group);
+cudaError_t launch_sba(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
+                       int avg_bits, const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, uint8_t* ws,
+                       DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev);
+cudaError_t launch_sqc(const float* W, int64_t m, int64_t n, const double* h, const uint8_t* bits, int group,
+                       int avg_bits, double lam, int n_tau, uint32_t* codes, float* scale, float* zero,
+                       uint8_t* tau_idx, int num_sms, cudaStream_t st);
+static std::atomic<long long> g_launches{0};
+void count_launches(int k) { g_launches.fetch_add(k, std::memory_order_relaxed); }
+}  // namespace slim
+
+using namespace slim;
+
+namespace {
+
+thread_local std::string g_last_cuda_error;
+constexpr double kDampAlpha = 0.01;
+constexpr size_t kStatusBytes = sizeof(DevStatus);
+constexpr int kMaxGroups = 1024;
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = cudaGetErrorString(e);
+  return SLIM_ECUDA;
+}
+
+#define SLIM_CUDA(call)                              \
+  do {                                               \
+    cudaError_t e__ = (call);                        \
+    if (e__ != cudaSuccess) return cuda_fail(e__);   \
+  } while (0)
+
+// Current device must be an sm_100 part; returns its SM count.
+int device_sms(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) { g_last_cuda_error = cudaGetErrorString(e); return SLIM_ENODEV; }
+  int major = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (major != 10) return SLIM_ENODEV;
+  cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev);
+  return SLIM_OK;
+}
+
+bool injected(const char* stage) {
+  const char* f = std::getenv("SLIM_FAULT");
+  return f && (std::strcmp(f, stage) == 0 || std::strcmp(f, "all") == 0);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int check_shape(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
+  if (m < 1 || n < 1 || N < 1) return SLIM_EINVAL;
+  if (group != 32 && group != 64 && group != 128) return SLIM_EINVAL;
+  if (n % group != 0) return SLIM_EINVAL;
+  if (n / group > kMaxGroups) return SLIM_EINVAL;
+  if (n > 65535 || m > (int64_t)1 << 30 || N > (int64_t)1 << 31) return SLIM_EINVAL;
+  if (xdtype != SLIM_X_F32 && xdtype != SLIM_X_BF16) return SLIM_EINVAL;
+  return SLIM_OK;
+}
+
+int check_bits(int avg_bits) { return (avg_bits >= 2 && avg_bits + 1 <= 8) ? SLIM_OK : SLIM_EINVAL; }
+
+// Sync the stream, then map CUDA errors and the device status word.
+int finish(cudaStream_t s, const DevStatus* dst) {
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  DevStatus hs;
+  e = cudaMemcpy(&hs, dst, sizeof(hs), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (hs.code == kStatusTimeout) return SLIM_ETIMEOUT;
+  if (hs.code == kStatusNotPD) return SLIM_ENOTPD;
+  if (hs.code == kStatusRangeCode) return SLIM_ERANGE;
+  if (hs.code != 0) return SLIM_ECUDA;
+  return SLIM_OK;
+}
+
+// Workspace holder: caller memory or a cudaMallocAsync'd block freed on scope exit.
+struct Workspace {
+  uint8_t* p = nullptr;
+  bool owned = false;
+  cudaStream_t s = nullptr;
+  int acquire(void* ws, size_t ws_bytes, size_t need, cudaStream_t st) {
+    s = st;
+    if (ws) {
+      if (ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255)) return SLIM_EINVAL;
+      p = static_cast<uint8_t*>(ws);
+      return SLIM_OK;
+    }
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&p), need, st);
+    if (e != cudaSuccess) { g_last_cuda_error = cudaGetErrorString(e); cudaGetLastError(); return SLIM_ENOMEM; }
+    owned = true;
+    return SLIM_OK;
+  }
+  ~Workspace() {
+    if (owned && p) { cudaFreeAsync(p, s); cudaStreamSynchronize(s); }
+  }
+};
+
+size_t hinv_bytes(int64_t n) { return hinv_workspace_doubles(n) * sizeof(double); }
+size_t sal_bytes(int64_t m, int64_t n) { return (size_t)salience_row_blocks(m) * n * sizeof(double); }
+
+// Layout of the full-path workspace.
+struct LayerWs {
+  size_t off_H, off_h, off_S, off_order, off_kl, off_pstar, off_scratch, total;
+};
+LayerWs layer_ws(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
+  LayerWs w{};
+  const int64_t k = n / group;
+  const int64_t P = k / 2 + 1;
+  size_t off = kStatusBytes;
+  w.off_H = off; off = al256(off + (size_t)n * n * 8);
+  w.off_h = off; off = al256(off + (size_t)n * 8);
+  w.off_S = off; off = al256(off + (size_t)k * 8);
+  w.off_order = off; off = al256(off + (size_t)k * 4);
+  w.off_kl = off; off = al256(off + (size_t)P * 8);
+  w.off_pstar = off; off = al256(off + 8);
+  size_t scratch = hessian_ws_bytes(N, n, xdtype);
+  size_t t = hinv_bytes(n); if (t > scratch) scratch = t;
+  t = sal_bytes(m, n); if (t > scratch) scratch = t;
+  t = sba_ws_bytes(m, n, N, xdtype, group); if (t > scratch) scratch = t;
+  w.off_scratch = off; off = al256(off + scratch);
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* slim_status_string(int status) {
+  switch (status) {
+    case SLIM_OK: return "ok";
+    case SLIM_EINVAL: return "invalid argument";
+    case SLIM_ENOMEM: return "out of device memory";
+    case SLIM_ECUDA: return "CUDA error";
+    case SLIM_ETIMEOUT: return "device wait timed out";
+    case SLIM_ENOTPD: return "damped Hessian is not positive definite";
+    case SLIM_ENODEV: return "no sm_100 device";
+    case SLIM_EINJECTED: return "injected failure";
+    case SLIM_ERANGE: return "a value is out of the fp16 operand range";
+    default: return "unknown status";
+  }
+}
+
+const char* slim_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
+const char* slim_version(void) { return "libslim 0.1 (sm_100a)"; }
+
+int slim_num_candidates(int64_t n, int group) {
+  if (group <= 0 || n % group) return -1;
+  return (int)(n / group / 2 + 1);
+}
+int64_t slim_row_words(int64_t n, int avg_bits) { return n * avg_bits / 32; }
+int64_t slim_launch_count(void) { return g_launches.load(); }
+
+// ------------------------------------------------------------------ hessian
+size_t slim_hessian_workspace_bytes(int64_t N, int64_t n, int xdtype) {
+  return kStatusBytes + al256(hessian_ws_bytes(N, n, xdtype));
+}
+
+int slim_hessian(const void* X, int xdtype, int64_t N, int64_t n, double* H, void* ws, size_t ws_bytes,
+                 void* stream) {
+  if (!X || !H || N < 1 || n < 32 || n % 32 || n > 65535 || (xdtype != 0 && xdtype != 1) || !aligned16(X))
+    return SLIM_EINVAL;
+  int sms = 0;
+  int rc = device_sms(&sms);
+  if (rc) return rc;
+  if (injected("hessian")) return SLIM_EINJECTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Workspace w;
+  rc = w.acquire(ws, ws_bytes, slim_hessian_workspace_bytes(N, n, xdtype), s);
+  if (rc) return rc;
+  DevStatus* st = reinterpret_cast<DevStatus*>(w.p);
+  SLIM_CUDA(cudaMemsetAsync(st, 0, kStatusBytes, s));
+  SLIM_CUDA(launch_hessian(X, xdtype, N, n, H, w.p + kStatusBytes, st, sms, s, nullptr));
+  return finish(s, st);
+}
+
+// ------------------------------------------------------------------ hinv_diag
+size_t slim_hinv_diag_workspace_bytes(int64_t n) { return kStatusBytes + al256(hinv_bytes(n)); }
+
+int slim_hinv_diag(const double* H, int64_t n, double alpha, double* h, void* ws, size_t ws_bytes, void* stream) {
+  if (!H || !h || n < 1 || n > 65535 || !(alpha >= 0.0)) return SLIM_EINVAL;
+  int sms = 0;
+  int rc = device_sms(&sms);
+  if (rc) return rc;
+  if (injected("hinv_diag")) return SLIM_EINJECTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Workspace w;
+  rc = w.acquire(ws, ws_bytes, slim_hinv_diag_workspace_bytes(n), s);
+  if (rc) return rc;
+  DevStatus* st = reinterpret_cast<DevStatus*>(w.p);
+  SLIM_CUDA(cudaMemsetAsync(st, 0, kStatusBytes, s));
+  SLIM_CUDA(launch_hinv(H, n, alpha, h, reinterpret_cast<double*>(w.p + kStatusBytes), st, s));
+  return finish(s, st);
+}
+
+// ------------------------------------------------------------------ salience
+size_t slim_salience_workspace_bytes(int64_t m, int64_t n, int group) {
+  (void)group;
+  return kStatusBytes + al256(sal_bytes(m, n));
+}
+
+int slim_salience(const float* W, int64_t m, int64_t n, const double* h, int group, double* S, int32_t* order,
+                  void* ws, size_t ws_bytes, void* stream) {
+  if (!W || !h || !S || !order || !aligned16(W)) return SLIM_EINVAL;
+  int rc = check_shape(m, n, 1, SLIM_X_BF16, group);
+  if (rc) return rc;
+  int sms = 0;
+  rc = device_sms(&sms);
+  if (rc) return rc;
+  if (injected("salience")) return SLIM_EINJECTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Workspace w;
+  rc = w.acquire(ws, ws_bytes, slim_salience_workspace_bytes(m, n, group), s);
+  if (rc) return rc;
+  DevStatus* st = reinterpret_cast<DevStatus*>(w.p);
+  SLIM_CUDA(cudaMemsetAsync(st, 0, kStatusBytes, s));
+  SLIM_CUDA(launch_salience(W, m, n, h, group, S, order, reinterpret_cast<double*>(w.p + kStatusBytes), s));
+  return finish(s, st);
+}
+
+// ------------------------------------------------------------------ sba_search
+size_t slim_sba_workspace_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
+  return kStatusBytes + al256(sba_ws_bytes(m, n, N, xdtype, group));
+}
+
+int slim_sba_search(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
+                    int avg_bits, const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, void* ws,
+                    size_t ws_bytes, void* stream) {
+  if (!W || !X || !order || !bits || !aligned16(W) || !aligned16(X)) return SLIM_EINVAL;
+  int rc = check_shape(m, n, N, xdtype, group);
+  if (rc) return rc;
+  rc = check_bits(avg_bits);
+  if (rc) return rc;
+  int sms = 0;
+  rc = device_sms(&sms);
+  if (rc) return rc;
+  if (injected("sba_search")) return SLIM_EINJECTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Workspace w;
+  rc = w.acquire(ws, ws_bytes, slim_sba_workspace_bytes(m, n, N, xdtype, group), s);
+  if (rc) return rc;
+  DevStatus* st = reinterpret_cast<DevStatus*>(w.p);
+  SLIM_CUDA(cudaMemsetAsync(st, 0, kStatusBytes, s));
+  SLIM_CUDA(launch_sba(W, m, n, X, xdtype, N, group, avg_bits, order, kl, p_star, bits, w.p + kStatusBytes, st,
+                       sms, s, nullptr));
+  return finish(s, st);
+}
+
+// ------------------------------------------------------------------ sqc
+int slim_sqc(const float* W, int64_t m, int64_t n, const double* h, const uint8_t* bits, int group, int avg_bits,
+             double lambda, int n_tau, uint32_t* codes, float* scale, float* zero, uint8_t* tau_idx,
+             void* stream) {
+  if (!W || !h || !bits || !codes || !scale || !zero) return SLIM_EINVAL;
+  int rc = check_shape(m, n, 1, SLIM_X_BF16, group);
+  if (rc) return rc;
+  rc = check_bits(avg_bits);
+  if (rc) return rc;
+  if (!(lambda >= 0.0 && lambda < 1.0) || n_tau < 1 || n_tau > 256) return SLIM_EINVAL;
+  int sms = 0;
+  rc = device_sms(&sms);
+  if (rc) return rc;
+  if (injected("sqc")) return SLIM_EINJECTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SLIM_CUDA(launch_sqc(W, m, n, h, bits, group, avg_bits, lambda, n_tau, codes, scale, zero, tau_idx, sms, s));
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SLIM_OK;
+}
+
+// ------------------------------------------------------------------ whole layer
+size_t slim_workspace_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group, int avg_bits) {
+  (void)avg_bits;
+  if (check_shape(m, n, N, xdtype, group)) return 0;
+  return layer_ws(m, n, N, xdtype, group).total;
+}
+
+int slim_quantize_layer_ex(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
+                           int avg_bits, double lambda, int n_tau, uint32_t* codes, float* scale, float* zero,
+                           uint8_t* bits, void* ws, size_t ws_bytes, void* stream, slim_diag* diag) {
+  if (!W || !X || !codes || !scale || !zero || !bits || !aligned16(W) || !aligned16(X)) return SLIM_EINVAL;
+  int rc = check_shape(m, n, N, xdtype, group);
+  if (rc) return rc;
+  rc = check_bits(avg_bits);
+  if (rc) return rc;
+  if (!(lambda >= 0.0 && lambda < 1.0) || n_tau < 1 || n_tau > 256) return SLIM_EINVAL;
+  int sms = 0;
+  rc = device_sms(&sms);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const LayerWs L = layer_ws(m, n, N, xdtype, group);
+  Workspace w;
+  rc = w.acquire(ws, ws_bytes, L.total, s);
+  if (rc) return rc;
+  DevStatus* st = reinterpret_cast<DevStatus*>(w.p);
+  double* H = (diag && diag->H) ? diag->H : reinterpret_cast<double*>(w.p + L.off_H);
+  double* h = (diag && diag->h) ? diag->h : reinterpret_cast<double*>(w.p + L.off_h);
+  double* S = (diag && diag->S) ? diag->S : reinterpret_cast<double*>(w.p + L.off_S);
+  int32_t* order = (diag && diag->order) ? diag->order : reinterpret_cast<int32_t*>(w.p + L.off_order);
+  double* kl = (diag && diag->kl) ? diag->kl : reinterpret_cast<double*>(w.p + L.off_kl);
+  int32_t* pstar = reinterpret_cast<int32_t*>(w.p + L.off_pstar);
+  uint8_t* tau = diag ? diag->tau_idx : nullptr;
+  uint8_t* scratch = w.p + L.off_scratch;
+
+  cudaEvent_t ev[10] = {};
+  const bool timed = diag != nullptr;
+  if (timed)
+    for (auto& e : ev) SLIM_CUDA(cudaEventCreate(&e));
+  cudaEvent_t* kev_h = timed ? ev + 6 : nullptr;
+  cudaEvent_t* kev_s = timed ? ev + 8 : nullptr;
+  auto rec = [&](int i) { if (timed) cudaEventRecord(ev[i], s); };
+  auto run = [&]() -> int {
+    SLIM_CUDA(cudaMemsetAsync(st, 0, kStatusBytes, s));
+    rec(0);
+    if (injected("hessian")) return SLIM_EINJECTED;
+    SLIM_CUDA(launch_hessian(X, xdtype, N, n, H, scratch, st, sms, s, kev_h));
+    rec(1);
+    if (injected("hinv_diag")) return SLIM_EINJECTED;
+    SLIM_CUDA(launch_hinv(H, n, kDampAlpha, h, reinterpret_cast<double*>(scratch), st, s));
+    rec(2);
+    if (injected("salience")) return SLIM_EINJECTED;
+    SLIM_CUDA(launch_salience(W, m, n, h, group, S, order, reinterpret_cast<double*>(scratch), s));
+    rec(3);
+    if (injected("sba_search")) return SLIM_EINJECTED;
+    SLIM_CUDA(launch_sba(W, m, n, X, xdtype, N, group, avg_bits, order, kl, pstar, bits, scratch, st, sms, s, kev_s));
+    rec(4);
+    if (injected("sqc")) return SLIM_EINJECTED;
+    SLIM_CUDA(launch_sqc(W, m, n, h, bits, group, avg_bits, lambda, n_tau, codes, scale, zero, tau, sms, s));
+    rec(5);
+    return finish(s, st);
+  };
+  rc = run();
+  if (timed) {
+    cudaStreamSynchronize(s);
+    if (rc == SLIM_OK) {
+      for (int i = 0; i < 5; ++i) cudaEventElapsedTime(&diag->stage_ms[i], ev[i], ev[i + 1]);
+      cudaEventElapsedTime(&diag->stage_ms[5], ev[0], ev[5]);
+      diag->stage_ms[6] = diag->stage_ms[7] = 0.f;
+      if (xdtype == SLIM_X_BF16) cudaEventElapsedTime(&diag->stage_ms[6], ev[6], ev[7]);
+      cudaEventElapsedTime(&diag->stage_ms[7], ev[8], ev[9]);
+      int32_t ps = -1;
+      cudaMemcpy(&ps, pstar, sizeof(ps), cudaMemcpyDeviceToHost);
+      diag->p_star = ps;
+    }
+    for (auto& e : ev) cudaEventDestroy(e);
+  }
+  return rc;
+}
+
+int slim_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
+                        int avg_bits, double lambda, int n_tau, uint32_t* codes, float* scale, float* zero,
+                        uint8_t* bits, void* ws, size_t ws_bytes, void* stream) {
+  return slim_quantize_layer_ex(W, m, n, X, xdtype, N, group, avg_bits, lambda, n_tau, codes, scale, zero, bits,
+                                ws, ws_bytes, stream, nullptr);
+}
+
+int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N,
+                             int group, int avg_bits, double lambda, int n_tau, uint32_t* codes, float* scale,
+                             float* zero, uint8_t* bits, void* stream) {
+  if (!W || !X || !codes || !scale || !zero || !bits) return SLIM_EINVAL;
+  int rc = check_shape(m, n, N, xdtype, group);
+  if (rc) return rc;
+  rc = check_bits(avg_bits);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t k = n / group;
+  const size_t wb = (size_t)m * n * 4, xb = (size_t)N * n * (xdtype == SLIM_X_BF16 ? 2 : 4);
+  const size_t cb = (size_t)m * slim_row_words(n, avg_bits) * 4, sb = (size_t)m * k * 4;
+  const LayerWs L = layer_ws(m, n, N, xdtype, group);
+  size_t off = 0;
+  const size_t o_w = off; off = al256(off + wb);
+  const size_t o_x = off; off = al256(off + xb);
+  const size_t o_c = off; off = al256(off + cb);
+  const size_t o_s = off; off = al256(off + sb);
+  const size_t o_z = off; off = al256(off + sb);
+  const size_t o_b = off; off = al256(off + (size_t)k);
+  const size_t o_ws = off; off = al256(off + L.total);
+  Workspace w;
+  rc = w.acquire(nullptr, 0, off, s);
+  if (rc) return rc;
+  SLIM_CUDA(cudaMemcpyAsync(w.p + o_w, W, wb, cudaMemcpyHostToDevice, s));
+  SLIM_CUDA(cudaMemcpyAsync(w.p + o_x, X, xb, cudaMemcpyHostToDevice, s));
+  rc = slim_quantize_layer(reinterpret_cast<const float*>(w.p + o_w), m, n, w.p + o_x, xdtype, N, group, avg_bits,
+                           lambda, n_tau, reinterpret_cast<uint32_t*>(w.p + o_c), reinterpret_cast<float*>(w.p + o_s),
+                           reinterpret_cast<float*>(w.p + o_z), w.p + o_b, w.p + o_ws, L.total, stream);
+  if (rc) return rc;
+  SLIM_CUDA(cudaMemcpyAsync(codes, w.p + o_c, cb, cudaMemcpyDeviceToHost, s));
+  SLIM_CUDA(cudaMemcpyAsync(scale, w.p + o_s, sb, cudaMemcpyDeviceToHost, s));
+  SLIM_CUDA(cudaMemcpyAsync(zero, w.p + o_z, sb, cudaMemcpyDeviceToHost, s));
+  SLIM_CUDA(cudaMemcpyAsync(bits, w.p + o_b, (size_t)k, cudaMemcpyDeviceToHost, s));
+  SLIM_CUDA(cudaStreamSynchronize(s));
+  return SLIM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,329 @@
+// hinv_diag: h_j = [H_d^-1]_jj, the inverse-Hessian diagonal of the salience
+// formula (SliM-LLM write-up, rkmt.cn, section 组件一 SBA).
+//
+// H_d = H with zero diagonal entries set to 1, plus alpha * mean(diag) on the
+// diagonal. With H_d = L L^T, H_d^-1 = L^-T L^-1, so h_j is the squared norm of
+// column j of M = L^-1. All arithmetic is fp64 on the CUDA cores, in 64 x 64
+// blocks (T = ceil(n / 64) block rows, the last one possibly 32 wide):
+//
+//   Cholesky, right-looking, per diagonal block K:
+//     potrf_diag   one CTA: L_KK = chol(A_KK) in shared memory, M_KK = L_KK^-1
+//     panel        L_IK = A_IK M_KK^T for every block row I > K
+//     syrk         A_IJ -= L_IK L_JK^T for K < J <= I (lower tiles only)
+//   Inverse, forward substitution of L M = I, right-looking, per block row I:
+//     rowmult      M_IJ = M_II R_IJ for J < I (R accumulates -sum L_IK M_KJ)
+//     update       R_I'J -= L_I'I M_IJ for I' > I, J <= I
+//   Column norms   h_j = sum_{i >= j} M_ij^2 (partials, then a fixed-order sum)
+//
+// Flops are n^3/3 for each half. A non-positive pivot records SLIM_ENOTPD with
+// its index; the remaining kernels run to completion on the bad values.
+#include <cstdint>
+#include "common.cuh"
+
+namespace slim {
+
+constexpr int NB = 64;
+constexpr int LDS = NB + 1;  // padded shared-memory row (doubles)
+
+// ---------------------------------------------------------------- damping
+__global__ void diag_sum_kernel(const double* __restrict__ H, int64_t n, double alpha, double* __restrict__ out) {
+  __shared__ double red[32];
+  double acc = 0.0;
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+    const double d = H[j * n + j];
+    acc += (d == 0.0) ? 1.0 : d;
+  }
+  acc = warp_sum(acc);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    double v = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.0;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) out[0] = alpha * (v / (double)n);
+  }
+}
+
+// A = lower triangle of H with the dead-column fix and damping; upper part 0.
+__global__ void damp_copy_kernel(const double* __restrict__ H, int64_t n, const double* __restrict__ damp,
+                                 double* __restrict__ A) {
+  const int64_t i = blockIdx.y;
+  const double dv = damp[0];
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n; j += (int64_t)gridDim.x * blockDim.x) {
+    double v = 0.0;
+    if (j < i) v = H[i * n + j];
+    else if (j == i) {
+      const double d = H[i * n + i];
+      v = ((d == 0.0) ? 1.0 : d) + dv;
+    }
+    A[i * n + j] = v;
+  }
+}
+
+// ---------------------------------------------------------------- tile helpers
+// Load a (rows x cols) block at G (row-major, leading dim ld) into S[64][LDS],
+// either as is (S[r][c] = G[r][c]) or transposed (S[c][r] = G[r][c]); zero fill.
+__device__ __forceinline__ void load_tile(double (*S)[LDS], const double* G, int64_t ld, int rows, int cols,
+                                          bool transpose) {
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+    const int r = e / NB, c = e % NB;
+    const double v = (r < rows && c < cols) ? G[(int64_t)r * ld + c] : 0.0;
+    if (transpose) S[c][r] = v; else S[r][c] = v;
+  }
+}
+
+// acc[r][c] = sum_l At[l][ty + 16 r] * B[l][tx + 16 c]   (256 threads)
+__device__ __forceinline__ void tile_mma(const double (*At)[LDS], const double (*B)[LDS], double (&acc)[4][4], int kdim) {
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = 0.0;
+  for (int l = 0; l < kdim; ++l) {
+    double a[4], b[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) a[r] = At[l][ty + 16 * r];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) b[c] = B[l][tx + 16 * c];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[r][c] = fma(a[r], b[c], acc[r][c]);
+  }
+}
+
+__host__ __device__ inline int blk_size(int64_t n, int b) {
+  const int64_t s = n - (int64_t)b * NB;
+  return (int)(s < NB ? s : NB);
+}
+
+// ---------------------------------------------------------------- Cholesky pieces
+// Factor diagonal block K of A in place; write M_KK = L_KK^-1 into M.
+__global__ void __launch_bounds__(256) potrf_diag_kernel(double* __restrict__ A, double* __restrict__ M, int64_t n,
+                                                         int K, DevStatus* st) {
+  extern __shared__ double smem[];
+  double (*s)[LDS] = reinterpret_cast<double (*)[LDS]>(smem);
+  double (*inv)[LDS] = reinterpret_cast<double (*)[LDS]>(smem + NB * LDS);
+  const int nb = blk_size(n, K);
+  const int64_t off = (int64_t)K * NB * n + (int64_t)K * NB;
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+    const int r = e / NB, c = e % NB;
+    s[r][c] = (r < nb && c < nb && c <= r) ? A[off + (int64_t)r * n + c] : 0.0;
+  }
+  __syncthreads();
+  for (int j = 0; j < nb; ++j) {
+    if (threadIdx.x == 0) {
+      const double d = s[j][j];
+      if (!(d > 0.0)) {
+        record_failure(st, kStatusNotPD, K * NB + j);
+        s[j][j] = 1.0;
+      } else {
+        s[j][j] = sqrt(d);
+      }
+    }
+    __syncthreads();
+    const double piv = s[j][j];
+    for (int i = j + 1 + threadIdx.x; i < nb; i += blockDim.x) s[i][j] = s[i][j] / piv;
+    __syncthreads();
+    const int rem = nb - j - 1;
+    for (int e = threadIdx.x; e < rem * rem; e += blockDim.x) {
+      const int i = j + 1 + e / rem, l = j + 1 + e % rem;
+      if (l <= i) s[i][l] = fma(-s[i][j], s[l][j], s[i][l]);
+    }
+    __syncthreads();
+  }
+  // inverse of the lower-triangular block, one column per thread (forward substitution)
+  if (threadIdx.x < NB) {
+    const int c = threadIdx.x;
+    for (int i = 0; i < NB; ++i) inv[i][c] = 0.0;
+    if (c < nb) {
+      for (int i = c; i < nb; ++i) {
+        double acc = (i == c) ? 1.0 : 0.0;
+        for (int l = c; l < i; ++l) acc = fma(-s[i][l], inv[l][c], acc);
+        inv[i][c] = acc / s[i][i];
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < nb * nb; e += blockDim.x) {
+    const int r = e / nb, c = e % nb;
+    A[off + (int64_t)r * n + c] = (c <= r) ? s[r][c] : 0.0;
+    M[off + (int64_t)r * n + c] = (c <= r) ? inv[r][c] : 0.0;
+  }
+}
+
+// L_IK = A_IK * M_KK^T for block rows I > K (one CTA per block row).
+__global__ void __launch_bounds__(256) panel_kernel(double* __restrict__ A, const double* __restrict__ M, int64_t n,
+                                                    int K) {
+  extern __shared__ double smem[];
+  double (*At)[LDS] = reinterpret_cast<double (*)[LDS]>(smem);
+  double (*Bs)[LDS] = reinterpret_cast<double (*)[LDS]>(smem + NB * LDS);
+  const int I = K + 1 + blockIdx.x;
+  const int nbk = blk_size(n, K), nbi = blk_size(n, I);
+  double* a = A + (int64_t)I * NB * n + (int64_t)K * NB;
+  const double* mk = M + (int64_t)K * NB * n + (int64_t)K * NB;
+  load_tile(At, a, n, nbi, nbk, true);   // At[l][r] = A_IK[r][l]
+  load_tile(Bs, mk, n, nbk, nbk, true);  // Bs[l][j] = M_KK[j][l]
+  __syncthreads();
+  double acc[4][4];
+  tile_mma(At, Bs, acc, nbk);
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int rr = ty + 16 * r, cc = tx + 16 * c;
+      if (rr < nbi && cc < nbk) a[(int64_t)rr * n + cc] = acc[r][c];
+    }
+}
+
+// lower-triangle tile index x -> (ti, tj), tj <= ti
+__device__ __forceinline__ void tri_index(int x, int& ti, int& tj) {
+  int t = (int)((sqrt(8.0 * (double)x + 1.0) - 1.0) * 0.5);
+  while ((t + 1) * (t + 2) / 2 <= x) ++t;
+  while (t * (t + 1) / 2 > x) --t;
+  ti = t;
+  tj = x - t * (t + 1) / 2;
+}
+
+// A_IJ -= L_IK L_JK^T for K < J <= I.
+__global__ void __launch_bounds__(256) syrk_kernel(double* __restrict__ A, int64_t n, int K) {
+  extern __shared__ double smem[];
+  double (*At)[LDS] = reinterpret_cast<double (*)[LDS]>(smem);
+  double (*Bs)[LDS] = reinterpret_cast<double (*)[LDS]>(smem + NB * LDS);
+  int ti, tj;
+  tri_index(blockIdx.x, ti, tj);
+  const int I = K + 1 + ti, J = K + 1 + tj;
+  const int nbk = blk_size(n, K), nbi = blk_size(n, I), nbj = blk_size(n, J);
+  load_tile(At, A + (int64_t)I * NB * n + (int64_t)K * NB, n, nbi, nbk, true);  // At[l][i] = L_IK[i][l]
+  load_tile(Bs, A + (int64_t)J * NB * n + (int64_t)K * NB, n, nbj, nbk, true);  // Bs[l][j] = L_JK[j][l]
+  __syncthreads();
+  double acc[4][4];
+  tile_mma(At, Bs, acc, nbk);
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  double* c0 = A + (int64_t)I * NB * n + (int64_t)J * NB;
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int rr = ty + 16 * r, cc = tx + 16 * c;
+      if (rr < nbi && cc < nbj && (I != J || cc <= rr)) c0[(int64_t)rr * n + cc] -= acc[r][c];
+    }
+}
+
+// ---------------------------------------------------------------- inverse pieces
+// M_IJ = M_II * R_IJ for J < I (one CTA per J), R_IJ stored in place.
+__global__ void __launch_bounds__(256) rowmult_kernel(double* __restrict__ M, int64_t n, int I) {
+  extern __shared__ double smem[];
+  double (*At)[LDS] = reinterpret_cast<double (*)[LDS]>(smem);
+  double (*Bs)[LDS] = reinterpret_cast<double (*)[LDS]>(smem + NB * LDS);
+  const int J = blockIdx.x;
+  const int nbi = blk_size(n, I), nbj = blk_size(n, J);
+  double* r = M + (int64_t)I * NB * n + (int64_t)J * NB;
+  load_tile(At, M + (int64_t)I * NB * n + (int64_t)I * NB, n, nbi, nbi, true);  // At[l][i] = M_II[i][l]
+  load_tile(Bs, r, n, nbi, nbj, false);                                            // Bs[l][j] = R_IJ[l][j]
+  __syncthreads();
+  double acc[4][4];
+  tile_mma(At, Bs, acc, nbi);
+  __syncthreads();
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int i = ty + 16 * rr, j = tx + 16 * c;
+      if (i < nbi && j < nbj) r[(int64_t)i * n + j] = acc[rr][c];
+    }
+}
+
+// R_I'J -= L_I'I M_IJ for I' > I, J <= I. Grid: (T - 1 - I) x (I + 1).
+__global__ void __launch_bounds__(256) inv_update_kernel(const double* __restrict__ L, double* __restrict__ M,
+                                                         int64_t n, int I) {
+  extern __shared__ double smem[];
+  double (*At)[LDS] = reinterpret_cast<double (*)[LDS]>(smem);
+  double (*Bs)[LDS] = reinterpret_cast<double (*)[LDS]>(smem + NB * LDS);
+  const int Ip = I + 1 + blockIdx.x, J = blockIdx.y;
+  const int nbi = blk_size(n, I), nbp = blk_size(n, Ip), nbj = blk_size(n, J);
+  load_tile(At, L + (int64_t)Ip * NB * n + (int64_t)I * NB, n, nbp, nbi, true);  // At[l][i'] = L_I'I[i'][l]
+  load_tile(Bs, M + (int64_t)I * NB * n + (int64_t)J * NB, n, nbi, nbj, false);  // Bs[l][j] = M_IJ[l][j]
+  __syncthreads();
+  double acc[4][4];
+  tile_mma(At, Bs, acc, nbi);
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  double* c0 = M + (int64_t)Ip * NB * n + (int64_t)J * NB;
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int i = ty + 16 * r, j = tx + 16 * c;
+      if (i < nbp && j < nbj) c0[(int64_t)i * n + j] -= acc[r][c];
+    }
+}
+
+// ---------------------------------------------------------------- column norms
+constexpr int kNormRows = 128;
+__global__ void colsumsq_partial_kernel(const double* __restrict__ M, int64_t n, double* __restrict__ part) {
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= n) return;
+  int64_t i0 = (int64_t)blockIdx.y * kNormRows;
+  int64_t i1 = i0 + kNormRows < n ? i0 + kNormRows : n;
+  if (i0 < j) i0 = j;
+  double acc = 0.0;
+  for (int64_t i = i0; i < i1; ++i) {
+    const double v = M[i * n + j];
+    acc = fma(v, v, acc);
+  }
+  part[(int64_t)blockIdx.y * n + j] = acc;
+}
+__global__ void colsumsq_final_kernel(const double* __restrict__ part, int nparts, int64_t n, double* __restrict__ h) {
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= n) return;
+  double acc = 0.0;
+  for (int p = 0; p < nparts; ++p) acc += part[(int64_t)p * n + j];
+  h[j] = acc;
+}
+
+size_t hinv_workspace_doubles(int64_t n) {
+  const int64_t parts = (n + kNormRows - 1) / kNormRows;
+  return (size_t)(2 * n * n + parts * n + 64);
+}
+
+cudaError_t launch_hinv(const double* H, int64_t n, double alpha, double* h, double* ws, DevStatus* st,
+                        cudaStream_t s) {
+  double* A = ws;
+  double* M = ws + n * n;
+  const int64_t parts = (n + kNormRows - 1) / kNormRows;
+  double* part = M + n * n;
+  double* damp = part + parts * n;
+  const size_t tile_smem = 2 * NB * LDS * sizeof(double);
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaFuncSetAttribute(potrf_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem);
+    cudaFuncSetAttribute(panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem);
+    cudaFuncSetAttribute(syrk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem);
+    cudaFuncSetAttribute(rowmult_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem);
+    cudaFuncSetAttribute(inv_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem);
+    attr_done = true;
+  }
+  diag_sum_kernel<<<1, 1024, 0, s>>>(H, n, alpha, damp);
+  damp_copy_kernel<<<dim3((unsigned)((n + 255) / 256), (unsigned)n), 256, 0, s>>>(H, n, damp, A);
+  cudaMemsetAsync(M, 0, (size_t)n * n * sizeof(double), s);
+  const int T = (int)((n + NB - 1) / NB);
+  for (int K = 0; K < T; ++K) {
+    potrf_diag_kernel<<<1, 256, tile_smem, s>>>(A, M, n, K, st);
+    const int below = T - 1 - K;
+    if (below > 0) {
+      panel_kernel<<<below, 256, tile_smem, s>>>(A, M, n, K);
+      syrk_kernel<<<below * (below + 1) / 2, 256, tile_smem, s>>>(A, n, K);
+    }
+  }
+  for (int I = 0; I < T; ++I) {
+    if (I > 0) rowmult_kernel<<<I, 256, tile_smem, s>>>(M, n, I);
+    if (I < T - 1) inv_update_kernel<<<dim3((unsigned)(T - 1 - I), (unsigned)(I + 1)), 256, tile_smem, s>>>(A, M, n, I);
+  }
+  colsumsq_partial_kernel<<<dim3((unsigned)((n + 255) / 256), (unsigned)parts), 256, 0, s>>>(M, n, part);
+  colsumsq_final_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, (int)parts, n, h);
+  count_launches(2 + T + 2 * (T - 1) + 2 * (T - 1) + 2);
+  return cudaGetLastError();
+}
+
+}  // namespace slim

@@ -1,0 +1,595 @@
+// sba_search: salience-determined bit allocation (SliM-LLM write-up, rkmt.cn,
+// section 组件一 SBA; atlas.scime.ai summary, section Approach).
+//
+// Candidate p promotes the p most salient groups to b+1 bits and demotes the p
+// least salient to b-1 bits, p = 0 .. k/2, and is scored by
+//   KL_p = mean_t KL(softmax(y_t) || softmax(yhat_t)),  y = X W^T, yhat = X W_p^T,
+// W_p the per-group min-max round-to-nearest dequantization under that
+// allocation. p* = the smallest p with the least KL.
+//
+// How all candidates are scored in one pass
+// -----------------------------------------
+// Write yhat_p = y + d_p with d_p = X (W_p - W)^T. Candidate p differs from p-1
+// in two groups only (the p-th most salient goes b -> b+1, the p-th least
+// salient b -> b-1), so
+//   d_0 = X E0^T,                        E0 = W^(b) - W
+//   d_p = d_{p-1} + X_{c+} Dp_{c+}^T + X_{c-} Dm_{c-}^T,
+//                                        Dp = W^(b+1) - W^(b), Dm = W^(b-1) - W^(b)
+// (the same sum, regrouped). Per token tile (128 tokens) and output tile (128
+// outputs), the tensor cores build y and d_0 in tensor memory (TMEM) from the
+// full K = n contraction, then add the two changed groups' K = 2g slices for
+// every further p. After each step the epilogue reads d_p from TMEM and
+// accumulates the softmax statistics. d carries the quantization error
+// directly (not as a difference of two large products). Operands are fp16
+// (11-bit significand): X converted from bf16 exactly, the weight-side arrays
+// scaled by 2^8 (exact) so small entries stay out of fp16 subnormals, and the
+// fp32 accumulators scaled back by 2^-8. Tensor-core work: 2Nnm (y) + 2Nnm
+// (d_0) + (P-1) 4Ngm (updates), instead of P 2Nnm for one dequant-GEMM per
+// candidate.
+//
+// KL from running sums, per token t and output range (with e_y = exp(y - M)):
+//   S_y = sum e_y, S_q = sum e_y exp(d), A = sum e_y d
+//   KL_t = log(S_q / S_y) - A / S_y        (= lse(y + d) - lse(y) - E_P[d])
+// The epilogue keeps e_y in TMEM in place of y after the first step, so later
+// steps need one exp per element.
+//
+// Kernels
+//   sba_prep       warp per (row, group): RTN at b-1, b, b+1 in fp64 (the
+//                  definition's operation order); writes fp16 2^8 W, E0, Dp, Dm
+//   x_to_f16       bf16 X -> fp16 (exact in fp16's normal range)
+//   x_split        fp32 X: X ~ X_hi + X_lo as two fp16 halves of X_cat
+//   sba_score      persistent tcgen05 kernel (below)
+//   sba_merge      per token: merges output-group partials in fp64 -> KL_t,
+//                  sums per token tile
+//   sba_final      KL_p = sum / N, p* = first argmin, bits
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include "common.cuh"
+#include "tmap.h"
+
+namespace slim {
+
+// ---------------------------------------------------------------- prep
+constexpr float kOpScale = 256.0f;          // weight-side operands are stored x 2^8
+constexpr float kOpUnscale = 1.0f / 256.0f;
+constexpr float kHalfMax = 65504.0f;
+constexpr int kStatusRange = kStatusRangeCode;
+
+__device__ __forceinline__ __half to_half_checked(float v, DevStatus* st, int where) {
+  if (!(fabsf(v) <= kHalfMax)) record_failure(st, kStatusRange, where);
+  return __float2half_rn(v);
+}
+
+template <int G>
+__global__ void __launch_bounds__(256) sba_prep_kernel(const float* __restrict__ W, int64_t m, int64_t n,
+                                                       int avg_bits, __half* __restrict__ Wb, __half* __restrict__ E0,
+                                                       __half* __restrict__ Dp, __half* __restrict__ Dm,
+                                                       DevStatus* st) {
+  constexpr int E = G / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t k = n / G;
+  const int64_t pairs = m * k;
+  const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t pr = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); pr < pairs; pr += wstride) {
+    const int64_t i = pr / k, c = pr - (pr / k) * k;
+    const int64_t base = i * n + c * G;
+    float w[E];
+    float lo = 0.f, hi = 0.f;
+#pragma unroll
+    for (int r = 0; r < E; ++r) {
+      w[r] = W[base + lane + 32 * r];
+      lo = r ? fminf(lo, w[r]) : w[r];
+      hi = r ? fmaxf(hi, w[r]) : w[r];
+    }
+    lo = warp_min(lo);
+    hi = warp_max(hi);
+    const double dlo = lo, dhi = hi;
+    const bool deg = (dhi == dlo);
+    double wh[3][E];
+#pragma unroll
+    for (int l = 0; l < 3; ++l) {
+      const int b = avg_bits - 1 + l;
+      const double qmax = (double)((1 << b) - 1);
+      const double s0 = deg ? 1.0 : (dhi - dlo) / qmax;
+      const double z0 = deg ? -dlo : -dlo / s0;
+#pragma unroll
+      for (int r = 0; r < E; ++r) {
+        double q = rint((double)w[r] / s0 + z0);
+        q = fmin(fmax(q, 0.0), qmax);
+        wh[l][r] = deg ? (double)w[r] : s0 * (q - z0);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < E; ++r) {
+      const int64_t o = base + lane + 32 * r;
+      const double wd = w[r];
+      Wb[o] = to_half_checked(w[r] * kOpScale, st, 300);
+      E0[o] = to_half_checked((float)(wh[1][r] - wd) * kOpScale, st, 301);
+      Dp[o] = to_half_checked((float)(wh[2][r] - wh[1][r]) * kOpScale, st, 302);
+      Dm[o] = to_half_checked((float)(wh[0][r] - wh[1][r]) * kOpScale, st, 303);
+    }
+  }
+}
+
+// bf16 -> fp16, 8 elements per thread (16-byte loads and stores).
+__global__ void x_to_f16_kernel(const uint4* __restrict__ X, int64_t n8, uint4* __restrict__ Y, DevStatus* st) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n8; e += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = X[e];
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[4];
+    bool bad = false;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float a = __uint_as_float(in[q] << 16), b = __uint_as_float(in[q] & 0xFFFF0000u);
+      bad |= !(fabsf(a) <= kHalfMax) || !(fabsf(b) <= kHalfMax);
+      const __half2 h = __floats2half2_rn(a, b);
+      out[q] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    if (bad) record_failure(st, kStatusRange, 310);
+    Y[e] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+__global__ void x_split_kernel(const float* __restrict__ X, int64_t N, int64_t n, __half* __restrict__ Xc,
+                               DevStatus* st) {
+  const int64_t total = N * n;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = e / n, j = e - t * n;
+    const float x = X[e];
+    const __half hi = to_half_checked(x, st, 311);
+    const __half lo = __float2half_rn(x - __half2float(hi));
+    Xc[t * 2 * n + j] = hi;
+    Xc[t * 2 * n + n + j] = lo;
+  }
+}
+
+// ---------------------------------------------------------------- scoring kernel
+constexpr int SB_BM = 128;        // tokens per tile (TMEM lanes)
+constexpr int SB_BN = 128;        // outputs per tile
+constexpr int SB_BK = 64;         // K elements per box (128 bytes of bf16)
+constexpr int SB_BOX = SB_BM * SB_BK * 2;  // 16 KB
+constexpr int SB_STAGE = 3 * SB_BOX;       // X, B1, B2
+constexpr int SB_GROUP_OUT = 2 * SB_BN;    // outputs per work unit (two TMEM slots)
+constexpr int SB_BAND = 32;                // token tiles per raster band
+constexpr int SB_MAX_K = 1024;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct SbaTmaps {
+  CUtensorMap x, wb, e0, dp, dm;
+};
+
+struct SbaParams {
+  int64_t N, m, n;
+  int g, k, P, ksplit;
+  int n_tt, n_og, n_ot;   // token tiles, output groups, output tiles
+  int stages;
+  const int32_t* order;
+  float* part;            // [n_tt][n_og][F][128], F = 2 + 2P
+  DevStatus* st;
+};
+
+struct Chunk {
+  int xcol, bcol, k16_lo, k16_hi;
+  int which;  // 0: phase A (Wb, E0); 1: Dp; 2: Dm
+};
+
+// Chunk list of item (p, s): returns the count; fills chunk c when idx == c.
+__device__ __forceinline__ int item_chunks(const SbaParams& p, const int32_t* order, int step, int idx, Chunk& ch) {
+  if (step == 0) {
+    const int kc_count = (int)((p.n + SB_BK - 1) / SB_BK);
+    const int cnt = kc_count * p.ksplit;
+    if (idx >= 0) {
+      const int kc = idx / p.ksplit, sx = idx - kc * p.ksplit;
+      ch.bcol = kc * SB_BK;
+      ch.xcol = ch.bcol + sx * (int)p.n;
+      ch.k16_lo = 0;
+      ch.k16_hi = 4;
+      ch.which = 0;
+    }
+    return cnt;
+  }
+  const int per_group = (p.g >= 64 ? p.g / 64 : 1) * p.ksplit;
+  const int cnt = 2 * per_group;
+  if (idx >= 0) {
+    const int gi = idx / per_group, rem = idx - gi * per_group;
+    const int c = gi == 0 ? order[step - 1] : order[p.k - step];
+    const int bx = rem / p.ksplit, sx = rem - bx * p.ksplit;
+    if (p.g >= 64) {
+      ch.bcol = c * p.g + 64 * bx;
+      ch.k16_lo = 0;
+      ch.k16_hi = 4;
+    } else {
+      const int col = c * p.g;
+      ch.bcol = (col / 64) * 64;
+      ch.k16_lo = (col % 64) / 16;
+      ch.k16_hi = ch.k16_lo + p.g / 16;
+    }
+    ch.xcol = ch.bcol + sx * (int)p.n;
+    ch.which = gi == 0 ? 1 : 2;
+  }
+  return cnt;
+}
+
+__device__ __forceinline__ void unit_decode(const SbaParams& p, int u, int& tt, int& og) {
+  const int band_start = (u / (SB_BAND * p.n_og)) * SB_BAND;
+  const int bc = (p.n_tt - band_start < SB_BAND) ? p.n_tt - band_start : SB_BAND;
+  const int r = u - band_start * p.n_og;
+  og = r / bc;
+  tt = band_start + (r - og * bc);
+}
+
+__global__ void __launch_bounds__(192, 1) sba_score_kernel(const __grid_constant__ SbaTmaps tm, SbaParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * SB_STAGE);
+  uint64_t* empty = full + S;
+  uint64_t* afull = empty + S;   // [2]
+  uint64_t* afree = afull + 2;   // [2]
+  uint64_t* done = afree + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  int32_t* s_order = reinterpret_cast<int32_t*>(tslot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int c = threadIdx.x; c < p.k; c += blockDim.x) s_order[c] = p.order[c];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&afull[s], 1); mbar_init(&afree[s], 4); }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, 512);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+  const int units = p.n_tt * p.n_og;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const void* bmaps[3][2] = {{&tm.wb, &tm.e0}, {&tm.dp, nullptr}, {&tm.dm, nullptr}};
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int tt, og;
+        unit_decode(p, u, tt, og);
+        const int nslots = (p.n_ot - 2 * og) < 2 ? (p.n_ot - 2 * og) : 2;
+        for (int step = 0; step < p.P && ok; ++step)
+          for (int s = 0; s < nslots && ok; ++s) {
+            Chunk ch;
+            const int nch = item_chunks(p, s_order, step, -1, ch);
+            const int brow = (og * 2 + s) * SB_BN;
+            for (int ci = 0; ci < nch; ++ci, ++it) {
+              item_chunks(p, s_order, step, ci, ch);
+              const int st = it % S;
+              const uint32_t ph = (it / S) & 1;
+              if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, p.st, 200 + st)) { ok = false; break; }
+              uint8_t* sb = smem + st * SB_STAGE;
+              const int nbox = ch.which == 0 ? 3 : 2;
+              mbar_arrive_expect_tx(&full[st], nbox * SB_BOX);
+              tma_load_2d(sb, &tm.x, &full[st], ch.xcol, tt * SB_BM);
+              tma_load_2d(sb + SB_BOX, bmaps[ch.which][0], &full[st], ch.bcol, brow);
+              if (ch.which == 0) tma_load_2d(sb + 2 * SB_BOX, bmaps[0][1], &full[st], ch.bcol, brow);
+            }
+          }
+      }
+      // let every issued copy land before the CTA can exit
+      for (uint32_t j = (it > (uint32_t)S ? it - S : 0); j < it; ++j) {
+        uint64_t t0 = global_ns();
+        while (!mbar_try_wait(&full[j % S], (j / S) & 1) && global_ns() - t0 < kWaitLimitNs) {}
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(SB_BM, SB_BN, false, false);
+      uint32_t it = 0;
+      uint32_t cnt[2] = {0, 0};
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int tt, og;
+        unit_decode(p, u, tt, og);
+        const int nslots = (p.n_ot - 2 * og) < 2 ? (p.n_ot - 2 * og) : 2;
+        for (int step = 0; step < p.P && ok; ++step)
+          for (int s = 0; s < nslots && ok; ++s) {
+            if (!mbar_wait(&afree[s], (cnt[s] & 1) ^ 1, abort_flag, p.st, 220 + s)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t ty = tbase + s * 256, td = ty + 128;
+            Chunk ch;
+            const int nch = item_chunks(p, s_order, step, -1, ch);
+            for (int ci = 0; ci < nch; ++ci, ++it) {
+              item_chunks(p, s_order, step, ci, ch);
+              const int st = it % S;
+              const uint32_t ph = (it / S) & 1;
+              if (!mbar_wait(&full[st], ph, abort_flag, p.st, 230 + st)) { ok = false; break; }
+              tc_fence_after();
+              const uint32_t xa = smem_u32(smem + st * SB_STAGE);
+              for (int k16 = ch.k16_lo; k16 < ch.k16_hi; ++k16) {
+                const uint64_t ad = sdesc_sw128(xa + k16 * 32, 16, 1024);
+                const uint64_t b1 = sdesc_sw128(xa + SB_BOX + k16 * 32, 16, 1024);
+                if (ch.which == 0) {
+                  const uint32_t acc = (ci > 0 || k16 > ch.k16_lo) ? 1u : 0u;
+                  const uint64_t b2 = sdesc_sw128(xa + 2 * SB_BOX + k16 * 32, 16, 1024);
+                  tc_mma_f16(ty, ad, b1, idesc, acc);
+                  tc_mma_f16(td, ad, b2, idesc, acc);
+                } else {
+                  tc_mma_f16(td, ad, b1, idesc, 1u);
+                }
+              }
+              tc_commit(&empty[st]);
+            }
+            if (!ok) break;
+            tc_commit(&afull[s]);
+            ++cnt[s];
+          }
+      }
+      tc_commit(done);
+      uint64_t t0 = global_ns();
+      while (!mbar_try_wait(done, 0) && global_ns() - t0 < kWaitLimitNs) {}
+    }
+  } else {
+    // ------------------------------------------------ epilogue: 4 warps, one token row per thread
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const int F = 2 + 2 * p.P;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    uint32_t cnt[2] = {0, 0};
+    bool ok = true;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      int tt, og;
+      unit_decode(p, u, tt, og);
+      const int nslots = (p.n_ot - 2 * og) < 2 ? (p.n_ot - 2 * og) : 2;
+      float* outp = p.part + ((size_t)tt * p.n_og + og) * F * SB_BM + r;
+      float Ms[2] = {0.f, 0.f}, Sys[2] = {0.f, 0.f}, fs[2] = {1.f, 1.f};
+      float sq_s0 = 0.f, a_s0 = 0.f;
+      for (int step = 0; step < p.P && ok; ++step)
+        for (int s = 0; s < nslots && ok; ++s) {
+          if (!mbar_wait(&afull[s], cnt[s] & 1, abort_flag, p.st, 240 + s)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t ty = tbase + lane_off + s * 256, td = ty + 128;
+          const int64_t col0 = (int64_t)(og * 2 + s) * SB_BN;
+          float sq = 0.f, a = 0.f;
+          if (step == 0) {
+            float mx = -3.0e38f;
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t yv[32];
+              tmem_ld32(ty + cc * 32, yv);
+              tc_wait_ld();
+#pragma unroll
+              for (int v = 0; v < 32; ++v)
+                if (col0 + cc * 32 + v < p.m) mx = fmaxf(mx, __uint_as_float(yv[v]) * kOpUnscale);
+            }
+            float sy = 0.f;
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t yv[32], dv[32];
+              tmem_ld32(ty + cc * 32, yv);
+              tmem_ld32(td + cc * 32, dv);
+              tc_wait_ld();
+#pragma unroll
+              for (int v = 0; v < 32; ++v) {
+                const bool valid = col0 + cc * 32 + v < p.m;
+                const float y = __uint_as_float(yv[v]) * kOpUnscale;
+                const float d = __uint_as_float(dv[v]) * kOpUnscale;
+                const float ey = valid ? exp2f((y - mx) * kLog2e) : 0.f;
+                sy += ey;
+                sq = fmaf(ey, exp2f(d * kLog2e), sq);
+                a = fmaf(ey, d, a);
+                yv[v] = __float_as_uint(ey);
+              }
+              tmem_st32(ty + cc * 32, yv);
+            }
+            tc_wait_st();
+            Ms[s] = mx;
+            Sys[s] = sy;
+          } else {
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t ev[32], dv[32];
+              tmem_ld32(ty + cc * 32, ev);
+              tmem_ld32(td + cc * 32, dv);
+              tc_wait_ld();
+#pragma unroll
+              for (int v = 0; v < 32; ++v) {
+                const float ey = __uint_as_float(ev[v]);
+                const float d = __uint_as_float(dv[v]) * kOpUnscale;
+                sq = fmaf(ey, exp2f(d * kLog2e), sq);
+                a = fmaf(ey, d, a);
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afree[s]);
+          ++cnt[s];
+          if (s == 0) { sq_s0 = sq; a_s0 = a; }
+          if (s == nslots - 1) {
+            if (step == 0) {
+              const float M = nslots == 2 ? fmaxf(Ms[0], Ms[1]) : Ms[0];
+              fs[0] = exp2f((Ms[0] - M) * kLog2e);
+              fs[1] = nslots == 2 ? exp2f((Ms[1] - M) * kLog2e) : 0.f;
+              outp[0] = M;
+              outp[SB_BM] = Sys[0] * fs[0] + (nslots == 2 ? Sys[1] * fs[1] : 0.f);
+            }
+            float sqt = sq_s0 * fs[0], at = a_s0 * fs[0];
+            if (nslots == 2) { sqt = fmaf(sq, fs[1], sqt); at = fmaf(a, fs[1], at); }
+            outp[(size_t)(2 + 2 * step) * SB_BM] = sqt;
+            outp[(size_t)(3 + 2 * step) * SB_BM] = at;
+          }
+        }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ---------------------------------------------------------------- merge and final
+__global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict__ part, int n_og, int P, int64_t N,
+                                                        int n_tt, double* __restrict__ kl_part) {
+  extern __shared__ float s_f[];  // [n_og][128] scale factors
+  __shared__ double red[4];
+  const int tt = blockIdx.x, r = threadIdx.x;
+  const int F = 2 + 2 * P;
+  const bool valid = (int64_t)tt * SB_BM + r < N;
+  const float* base = part + (size_t)tt * n_og * F * SB_BM + r;
+  float M = -3.0e38f;
+  for (int og = 0; og < n_og; ++og) M = fmaxf(M, base[(size_t)og * F * SB_BM]);
+  double Sy = 0.0;
+  for (int og = 0; og < n_og; ++og) {
+    const float f = exp2f((base[(size_t)og * F * SB_BM] - M) * kLog2e);
+    s_f[og * SB_BM + r] = f;
+    Sy += (double)base[(size_t)og * F * SB_BM + SB_BM] * (double)f;
+  }
+  for (int q = 0; q < P; ++q) {
+    double sq = 0.0, a = 0.0;
+    for (int og = 0; og < n_og; ++og) {
+      const double f = s_f[og * SB_BM + r];
+      sq += (double)base[((size_t)og * F + 2 + 2 * q) * SB_BM] * f;
+      a += (double)base[((size_t)og * F + 3 + 2 * q) * SB_BM] * f;
+    }
+    double kl = valid ? (log(sq / Sy) - a / Sy) : 0.0;
+    kl = warp_sum(kl);
+    if ((r & 31) == 0) red[r >> 5] = kl;
+    __syncthreads();
+    if (r == 0) kl_part[(size_t)q * n_tt + tt] = (red[0] + red[1]) + (red[2] + red[3]);
+    __syncthreads();
+  }
+}
+
+__global__ void sba_final_kernel(const double* __restrict__ kl_part, int n_tt, int P, int64_t N,
+                                 const int32_t* __restrict__ order, int k, int avg_bits, double* __restrict__ kl_out,
+                                 int32_t* __restrict__ pstar_out, uint8_t* __restrict__ bits) {
+  __shared__ double s_kl[SB_MAX_K / 2 + 1];
+  __shared__ int s_p;
+  for (int q = threadIdx.x; q < P; q += blockDim.x) {
+    double acc = 0.0;
+    for (int t = 0; t < n_tt; ++t) acc += kl_part[(size_t)q * n_tt + t];
+    s_kl[q] = acc / (double)N;
+    if (kl_out) kl_out[q] = s_kl[q];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int best = 0;
+    for (int q = 1; q < P; ++q)
+      if (s_kl[q] < s_kl[best]) best = q;
+    s_p = best;
+    if (pstar_out) *pstar_out = best;
+  }
+  __syncthreads();
+  const int ps = s_p;
+  for (int c = threadIdx.x; c < k; c += blockDim.x) bits[c] = (uint8_t)avg_bits;
+  __syncthreads();
+  for (int q = threadIdx.x; q < ps; q += blockDim.x) {
+    bits[order[q]] = (uint8_t)(avg_bits + 1);
+    bits[order[k - 1 - q]] = (uint8_t)(avg_bits - 1);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+struct SbaPlan {
+  int k, P, ksplit, n_tt, n_og, n_ot, stages;
+  size_t off_wb, off_e0, off_dp, off_dm, off_xc, off_part, off_klp, total;
+  size_t smem;
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+SbaPlan sba_plan(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
+  SbaPlan pl{};
+  pl.k = (int)(n / group);
+  pl.P = pl.k / 2 + 1;
+  pl.ksplit = xdtype == 1 ? 1 : 2;
+  pl.n_tt = (int)((N + SB_BM - 1) / SB_BM);
+  pl.n_ot = (int)((m + SB_BN - 1) / SB_BN);
+  pl.n_og = (pl.n_ot + 1) / 2;
+  const size_t wbytes = (size_t)m * n * 2;
+  size_t off = 0;
+  pl.off_wb = off; off = align256(off + wbytes);
+  pl.off_e0 = off; off = align256(off + wbytes);
+  pl.off_dp = off; off = align256(off + wbytes);
+  pl.off_dm = off; off = align256(off + wbytes);
+  pl.off_xc = off; off = align256(off + (size_t)N * pl.ksplit * n * 2);
+  pl.off_part = off; off = align256(off + (size_t)pl.n_tt * pl.n_og * (2 + 2 * pl.P) * SB_BM * sizeof(float));
+  pl.off_klp = off; off = align256(off + (size_t)pl.P * pl.n_tt * sizeof(double));
+  pl.total = off;
+  const size_t fixed = 1024 + 256 + (size_t)pl.k * 4 + 64;
+  int st = 4;
+  while (st > 2 && fixed + (size_t)st * SB_STAGE > 227 * 1024) --st;
+  pl.stages = st;
+  pl.smem = fixed + (size_t)st * SB_STAGE;
+  // more than half of the SM's shared memory: one CTA per SM, so the 512-column
+  // TMEM allocation never waits on a second resident CTA
+  if (pl.smem < 120 * 1024) pl.smem = 120 * 1024;
+  return pl;
+}
+
+size_t sba_ws_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
+  return sba_plan(m, n, N, xdtype, group).total;
+}
+
+cudaError_t launch_sba(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
+                       int avg_bits, const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, uint8_t* ws,
+                       DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev) {
+  const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
+  if (pl.k > SB_MAX_K) return cudaErrorInvalidValue;
+  __half* Wb = reinterpret_cast<__half*>(ws + pl.off_wb);
+  __half* E0 = reinterpret_cast<__half*>(ws + pl.off_e0);
+  __half* Dp = reinterpret_cast<__half*>(ws + pl.off_dp);
+  __half* Dm = reinterpret_cast<__half*>(ws + pl.off_dm);
+  __half* Xc = reinterpret_cast<__half*>(ws + pl.off_xc);
+  float* part = reinterpret_cast<float*>(ws + pl.off_part);
+  double* klp = reinterpret_cast<double*>(ws + pl.off_klp);
+
+  const int64_t pairs = m * pl.k;
+  int pgrid = (int)((pairs + 7) / 8);
+  if (pgrid > num_sms * 16) pgrid = num_sms * 16;
+  switch (group) {
+    case 32: sba_prep_kernel<32><<<pgrid, 256, 0, s>>>(W, m, n, avg_bits, Wb, E0, Dp, Dm, st); break;
+    case 64: sba_prep_kernel<64><<<pgrid, 256, 0, s>>>(W, m, n, avg_bits, Wb, E0, Dp, Dm, st); break;
+    case 128: sba_prep_kernel<128><<<pgrid, 256, 0, s>>>(W, m, n, avg_bits, Wb, E0, Dp, Dm, st); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (pl.ksplit == 2) {
+    x_split_kernel<<<num_sms * 8, 256, 0, s>>>(static_cast<const float*>(X), N, n, Xc, st);
+  } else {
+    x_to_f16_kernel<<<num_sms * 8, 256, 0, s>>>(static_cast<const uint4*>(X), N * n / 8, reinterpret_cast<uint4*>(Xc), st);
+  }
+  const void* xptr = Xc;
+  SbaTmaps tm;
+  bool ok = make_tmap_f16(&tm.x, xptr, (uint64_t)(n * pl.ksplit), (uint64_t)N, SB_BK, SB_BM);
+  ok = ok && make_tmap_f16(&tm.wb, Wb, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
+  ok = ok && make_tmap_f16(&tm.e0, E0, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
+  ok = ok && make_tmap_f16(&tm.dp, Dp, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
+  ok = ok && make_tmap_f16(&tm.dm, Dm, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
+  if (!ok) return cudaErrorInvalidValue;
+
+  SbaParams p;
+  p.N = N; p.m = m; p.n = n; p.g = group; p.k = pl.k; p.P = pl.P; p.ksplit = pl.ksplit;
+  p.n_tt = pl.n_tt; p.n_og = pl.n_og; p.n_ot = pl.n_ot; p.stages = pl.stages;
+  p.order = order; p.part = part; p.st = st;
+  cudaError_t e = cudaFuncSetAttribute(sba_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
+  if (e != cudaSuccess) return e;
+  const int units = pl.n_tt * pl.n_og;
+  const int grid = units < num_sms ? units : num_sms;
+  if (kev) cudaEventRecord(kev[0], s);
+  sba_score_kernel<<<grid, 192, pl.smem, s>>>(tm, p);
+  if (kev) cudaEventRecord(kev[1], s);
+  const size_t msmem = (size_t)pl.n_og * SB_BM * sizeof(float);
+  if (msmem > 48 * 1024) {
+    e = cudaFuncSetAttribute(sba_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+    if (e != cudaSuccess) return e;
+  }
+  sba_merge_kernel<<<pl.n_tt, SB_BM, msmem, s>>>(part, pl.n_og, pl.P, N, pl.n_tt, klp);
+  sba_final_kernel<<<1, 256, 0, s>>>(klp, pl.n_tt, pl.P, N, order, pl.k, avg_bits, kl, p_star, bits);
+  count_launches(5);
+  return cudaGetLastError();
+}
+
+}  // namespace slim

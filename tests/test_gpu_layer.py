@@ -1,0 +1,123 @@
+"""End-to-end GPU parity of slim_quantize_layer_ex through the C ABI.
+
+Each stage's output is checked against the oracle step fed with the GPU's own
+upstream outputs (identical inputs, so decisions must agree exactly), and the
+GPU's intermediate values against the oracle's full pipeline within the stated
+tolerances (decisions equal unless the oracle shows a near tie).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import slim_oracle as O
+from post_weight_quantization_hessian_b200 import slim
+from post_weight_quantization_hessian_b200 import synthetic as syn
+import json
+import os
+
+from parity_util import KL_ATOL, compare_sqc, device_inputs, hessian_bound, order_ok, pstar_ok, x_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def run_and_compare(s: syn.LayerSpec, h_rtol):
+    W, Xh, Wd, Xd = device_inputs(s)
+    X = x_f64(s, Xh)
+    d = slim.slim_quantize_layer_ex(Wd, Xd, s.group, s.avg_bits, s.lam, s.n_tau)
+    g = {k: (v.cpu().numpy() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    ref = O.quantize_layer(W, X, s.group, s.avg_bits, s.lam, s.n_tau)
+    # hessian and inverse diagonal vs the oracle pipeline
+    scale = 2.0 * (np.abs(X).T @ np.abs(X))
+    assert np.all(np.abs(g["H"] - ref.H) <= hessian_bound(s.N) * scale + 1e-300)
+    np.testing.assert_allclose(g["h"], ref.h, rtol=h_rtol)
+    # stage-by-stage on the GPU's own upstream values
+    np.testing.assert_allclose(g["h"], O.hinv_diag(g["H"]), rtol=1e-9)
+    S_chain = O.group_salience(W, g["h"], s.group)
+    np.testing.assert_allclose(g["S"], S_chain, rtol=1e-12)
+    assert order_ok(g["order"], S_chain, rel=1e-12) == 0
+    mism = order_ok(g["order"], ref.S, rel=1e-5)               # vs the pipeline: near ties only
+    sba_chain = O.sba_search(W, X, g["order"], s.group, s.avg_bits)
+    assert np.abs(g["kl"] - sba_chain.kl).max() <= KL_ATOL
+    if pstar_ok(g["p_star"], sba_chain.kl):
+        assert np.array_equal(g["bits"], sba_chain.bits.astype(np.uint8))
+    assert g["bits"].astype(int).sum() == s.k * s.avg_bits
+    sqc_chain = O.sqc_calibrate(W, g["h"], g["bits"], s.group, s.lam, s.n_tau)
+    agree, tmis = compare_sqc(g["codes"], g["scale"], g["zero"], g["tau_idx"], sqc_chain, g["bits"], s.group,
+                              s.avg_bits)
+    assert agree >= 0.9999 and tmis == 0
+    print(f"{s.name}: p* {g['p_star']} (oracle {ref.sba.p_star}, margin {ref.sba.margin:.2e}); order mismatches "
+          f"vs pipeline {mism}; KL {g['kl']} vs {ref.sba.kl}; stage ms {g['stage_ms']}")
+    return g, ref
+
+
+def test_tiny_layer_f32():
+    g, ref = run_and_compare(syn.TINY, h_rtol=1e-10)
+    assert g["p_star"] == ref.sba.p_star
+    assert np.array_equal(g["order"], ref.order)
+    assert np.array_equal(g["tau_idx"], ref.sqc.tau_idx)
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(group=64, avg_bits=3, N=3000), dict(group=32, m=384, n=256)])
+def test_small_layer_bf16(kw):
+    base = dict(name="small_bf16", m=320, n=768, N=1500, x_dtype="bf16", group=128, avg_bits=2, seed=9,
+                n_w_salient=8, w_scale=6.0, n_x_outliers=3, x_scale=25.0)
+    base.update(kw)
+    run_and_compare(syn.LayerSpec(**base), h_rtol=1e-3)
+
+
+def test_full_size_q_proj_sampled():
+    """LLaMA-7B q_proj shape, 262144 bf16 tokens, the launch configuration bench.py times."""
+    s = syn.Q_PROJ_7B
+    W, Xh, Wd, Xd = device_inputs(s)
+    d = slim.slim_quantize_layer_ex(Wd, Xd, s.group, s.avg_bits, s.lam, s.n_tau)
+    g = {k: (v.cpu().numpy() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    rng = np.random.default_rng(0)
+    # H on sampled columns (outlier and cluster columns included)
+    cols = np.unique(np.concatenate([syn.outlier_columns(s), syn.salient_columns(s)[::8],
+                                     rng.choice(s.n, 24, replace=False)]))
+    Xs = syn.bf16_bits_to_f32(Xh[:, cols]).astype(np.float64)
+    Hs = O.hessian(Xs)
+    scale = 2.0 * (np.abs(Xs).T @ np.abs(Xs))
+    err = np.abs(g["H"][np.ix_(cols, cols)] - Hs) / scale
+    print(f"full-size H sampled max rel-to-abs-sum error {err.max():.2e}")
+    assert err.max() <= hessian_bound(s.N)
+    # inverse diagonal and salience on the GPU's own H
+    np.testing.assert_allclose(g["h"], O.hinv_diag(g["H"]), rtol=1e-9)
+    S_chain = O.group_salience(W, g["h"], s.group)
+    np.testing.assert_allclose(g["S"], S_chain, rtol=1e-12)
+    assert order_ok(g["order"], S_chain, rel=1e-12) == 0
+    # the three salient clusters lead the order
+    lead = set(g["order"][:3].tolist())
+    assert lead == set((np.array(syn.LLAMA7B_CLUSTER_STARTS) // s.group).tolist())
+    # KL on a token subset, same kernels, oracle exact
+    sub = 4096
+    kl_s, p_s, bits_s = slim.slim_sba_search(Wd, Xd[:sub].contiguous(), s.group, s.avg_bits,
+                                             torch.from_numpy(g["order"]).cuda())
+    Xsub = syn.bf16_bits_to_f32(Xh[:sub]).astype(np.float64)
+    ref_s = O.sba_search(W, Xsub, g["order"], s.group, s.avg_bits, reassociate=True)
+    dev = np.abs(kl_s.cpu().numpy() - ref_s.kl).max()
+    print(f"full-size subset KL max |dKL| {dev:.2e}; p* {int(p_s.item())} vs {ref_s.p_star}")
+    assert dev <= KL_ATOL
+    pstar_ok(int(p_s.item()), ref_s.kl)
+    # full-N decisions against the oracle's stored values (tests/golden, written by make_golden.py)
+    gold = json.load(open(os.path.join(os.path.dirname(__file__), "golden", f"{s.name}.json")))
+    S_gold = np.array(gold["S"])
+    np.testing.assert_allclose(g["S"], S_gold, rtol=1e-4)
+    mism = order_ok(g["order"], S_gold, rel=1e-5)
+    assert np.abs(g["kl"] - np.array(gold["kl"])).max() <= KL_ATOL
+    assert g["p_star"] == gold["p_star"]
+    assert g["bits"].astype(int).tolist() == gold["bits"]
+    print(f"full-size vs golden: order mismatches {mism} (near ties only), max |dKL| "
+          f"{np.abs(g['kl'] - np.array(gold['kl'])).max():.2e}, p* {g['p_star']}")
+    # full-N search: invariants
+    kl = g["kl"]
+    assert np.all(kl >= 0) and g["p_star"] == int(np.argmin(kl))
+    b = g["bits"].astype(int)
+    assert b.sum() == s.k * s.avg_bits and (b == 3).sum() == (b == 1).sum() == g["p_star"]
+    # SQC on sampled rows with the GPU's h and bits
+    rows = np.sort(rng.choice(s.m, 64, replace=False))
+    ref_q = O.sqc_calibrate(W[rows], g["h"], g["bits"], s.group, s.lam, s.n_tau)
+    agree, tmis = compare_sqc(g["codes"][rows], g["scale"][rows], g["zero"][rows], g["tau_idx"][rows], ref_q,
+                              g["bits"], s.group, s.avg_bits)
+    assert agree >= 0.9999 and tmis == 0
+    print(f"full-size: p* {g['p_star']}, KL {kl}, stage ms {g['stage_ms']}")
