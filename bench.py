@@ -72,6 +72,9 @@ class ClockSampler:
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 3.0:     # first sample before the timed region
+                time.sleep(0.05)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
@@ -346,7 +349,7 @@ def run_ours(args, spec, world, rank, local):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=syn.Q_PROJ_7B.name, choices=sorted(syn.WORKLOADS))
@@ -354,9 +357,12 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=2048)
     ap.add_argument("--ref-rows", type=int, default=128)
+    ap.add_argument("--tokens", type=int, default=0, help="override N (profiling runs on a smaller case)")
     args = ap.parse_args(argv)
     world, rank, local = dist_setup(args)
     spec = syn.WORKLOADS[args.workload]
+    if args.tokens:
+        spec = spec.replace(N=args.tokens)
     try:
         if args.impl == "reference":
             return run_reference(args, spec, world, rank)

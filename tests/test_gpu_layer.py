@@ -102,7 +102,9 @@ def test_full_size_q_proj_sampled():
     # full-N decisions against the oracle's stored values (tests/golden, written by make_golden.py)
     gold = json.load(open(os.path.join(os.path.dirname(__file__), "golden", f"{s.name}.json")))
     S_gold = np.array(gold["S"])
-    np.testing.assert_allclose(g["S"], S_gold, rtol=1e-4)
+    # the truncating tensor-core accumulation scales H by up to hessian_bound; h and so
+    # S inherit about twice that relative shift, nearly uniform across groups
+    np.testing.assert_allclose(g["S"], S_gold, rtol=2 * hessian_bound(s.N))
     mism = order_ok(g["order"], S_gold, rel=1e-5)
     assert np.abs(g["kl"] - np.array(gold["kl"])).max() <= KL_ATOL
     assert g["p_star"] == gold["p_star"]
