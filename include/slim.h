@@ -116,6 +116,25 @@ int slim_salience(const float* W, int64_t m, int64_t n, const double* h, int gro
                   double* S, int32_t* order, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * slim_salience_noalloc: the same computation and outputs as slim_salience,
+ * for callers that cannot allocate device memory. The pages have no
+ * counterpart; it is a deployment variant. Some callers may not call
+ * cudaMalloc or let a library do so: code that runs inside an engine that owns
+ * every byte of device memory through its own pool and budget, code on a path
+ * where the implicit device synchronization of cudaMalloc/cudaFree is not
+ * acceptable, or code under a fixed memory cap planned in advance. This entry
+ * point allocates nothing: its scratch is a fixed 256 KiB device array inside
+ * the library (held on every GPU that loads the library until the process
+ * exits), enough for n <= 32768 input columns; larger n returns SLIM_EINVAL.
+ * The first call on a device looks up that array's device address, so make a
+ * first call on each device before any stream capture. All calls on a device
+ * share the array: calls that overlap on the GPU race and must be serialized
+ * by the caller. The call waits for `stream` to drain before returning.
+ */
+int slim_salience_noalloc(const float* W, int64_t m, int64_t n, const double* h, int group,
+                          double* S, int32_t* order, void* stream);
+
+/* ------------------------------------------------------------------------
  * slim_sba_search: salience-determined bit allocation ([P1] 组件一 SBA,
  * [P2] Approach). For p = 0 .. floor(k/2): groups order[0..p) get avg_bits+1,
  * groups order[k-p..k) get avg_bits-1, the rest avg_bits (balanced counts, so

@@ -13,7 +13,9 @@
 //   rank_sort      one block: rank_c = #{c' : S_c' > S_c or (S_c' == S_c and
 //                  c' < c)}, a stable descending order.
 #include <cstdint>
+#include <mutex>
 #include "common.cuh"
+#include "../../include/slim.h"
 
 namespace slim {
 
@@ -90,3 +92,95 @@ cudaError_t launch_salience(const float* W, int64_t m, int64_t n, const double* 
 }
 
 }  // namespace slim
+
+namespace slim {
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant (slim_salience_noalloc).
+//
+// Its scratch, the per-row-block column sums of squares, lives in one fixed
+// file-scope device array instead of caller or library allocations. Every GPU
+// that loads the library holds these 256 KiB until the process exits, and all
+// calls on a device share them: calls that overlap on the GPU race. The array
+// is fully rewritten by each call before it is read, so nothing carries over.
+// ---------------------------------------------------------------------------
+constexpr int64_t kNoAllocScratchDoubles = 32768;  // 256 KiB: row blocks x n <= 32768
+static __device__ __align__(256) double g_salience_scratch[kNoAllocScratchDoubles];
+
+// Column sums of squares over runs of `rows_per_block` rows (runtime), the
+// same per-thread arithmetic as colsq_partial_kernel.
+__global__ void __launch_bounds__(kColThreads)
+colsq_partial_rows_kernel(const float* __restrict__ W, int64_t m, int64_t n, int64_t rows_per_block,
+                          double* __restrict__ part) {
+  const int64_t col = ((int64_t)blockIdx.x * kColThreads + threadIdx.x) * 4;
+  const int64_t r0 = (int64_t)blockIdx.y * rows_per_block;
+  if (col >= n) return;
+  const int64_t r1 = (r0 + rows_per_block < m) ? r0 + rows_per_block : m;
+  double a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+  const float4* p = reinterpret_cast<const float4*>(W + r0 * n + col);
+  const int64_t stride = n / 4;
+  for (int64_t r = r0; r < r1; ++r, p += stride) {
+    const float4 v = *p;
+    a0 += (double)v.x * (double)v.x;
+    a1 += (double)v.y * (double)v.y;
+    a2 += (double)v.z * (double)v.z;
+    a3 += (double)v.w * (double)v.w;
+  }
+  double* o = part + (int64_t)blockIdx.y * n + col;
+  o[0] = a0; o[1] = a1; o[2] = a2; o[3] = a3;
+}
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+double* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_salience_scratch on the current device, looked up once
+// per device (host code cannot use the array's name as a device pointer).
+cudaError_t noalloc_scratch(double** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_salience_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = static_cast<double*>(p);
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+}  // namespace slim
+
+extern "C" int slim_salience_noalloc(const float* W, int64_t m, int64_t n, const double* h, int group, double* S,
+                                     int32_t* order, void* stream) {
+  using namespace slim;
+  if (!W || !h || !S || !order || (reinterpret_cast<uintptr_t>(W) & 15)) return SLIM_EINVAL;
+  if (m < 1 || n < 1 || (group != 32 && group != 64 && group != 128) || n % group || n / group > 1024)
+    return SLIM_EINVAL;
+  if (n > kNoAllocScratchDoubles) return SLIM_EINVAL;  // beyond the fixed scratch: at most 32768 input columns
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SLIM_ENODEV;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (major != 10) return SLIM_ENODEV;
+  double* part = nullptr;
+  if (noalloc_scratch(&part) != cudaSuccess) return SLIM_ECUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int64_t rb = (m + kRowsPerBlock - 1) / kRowsPerBlock;
+  if (rb > kNoAllocScratchDoubles / n) rb = kNoAllocScratchDoubles / n;
+  const int64_t rows_per_block = (m + rb - 1) / rb;
+  rb = (m + rows_per_block - 1) / rows_per_block;
+  dim3 g1((unsigned)((n / 4 + kColThreads - 1) / kColThreads), (unsigned)rb);
+  colsq_partial_rows_kernel<<<g1, kColThreads, 0, st>>>(W, m, n, rows_per_block, part);
+  const int k = (int)(n / group);
+  group_reduce_kernel<<<k, 256, 0, st>>>(part, (int)rb, m, n, h, group, S);
+  rank_sort_kernel<<<1, 1024, 0, st>>>(S, k, order);
+  count_launches(3);
+  if (cudaGetLastError() != cudaSuccess) return SLIM_ECUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SLIM_ECUDA;
+  return SLIM_OK;
+}

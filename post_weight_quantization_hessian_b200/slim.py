@@ -54,6 +54,7 @@ _SIGS = {
     "slim_hinv_diag": (i32, [vp, i64, dbl, vp, vp, sz, vp]),
     "slim_salience_workspace_bytes": (sz, [i64, i64, i32]),
     "slim_salience": (i32, [vp, i64, i64, vp, i32, vp, vp, vp, sz, vp]),
+    "slim_salience_noalloc": (i32, [vp, i64, i64, vp, i32, vp, vp, vp]),
     "slim_sba_workspace_bytes": (sz, [i64, i64, i64, i32, i32]),
     "slim_sba_search": (i32, [vp, i64, i64, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp]),
     "slim_sqc": (i32, [vp, i64, i64, vp, vp, i32, i32, dbl, i32, vp, vp, vp, vp, vp]),
@@ -180,6 +181,19 @@ def slim_salience(W: torch.Tensor, h: torch.Tensor, group: int, S=None, order=No
     wsb = ws.numel() * ws.element_size() if isinstance(ws, torch.Tensor) else 0
     _check(_lib().slim_salience(_ptr(W), m, n, _ptr(h), group, _ptr(S), _ptr(order), _ptr(ws), wsb,
                                 _stream(stream)), "slim_salience")
+    return S, order
+
+
+def slim_salience_noalloc(W: torch.Tensor, h: torch.Tensor, group: int, S=None, order=None, stream=None):
+    """slim_salience without any device allocation by the library (fixed internal scratch)."""
+    m, n = W.shape
+    k = n // group
+    if S is None:
+        S = torch.empty(k, dtype=torch.float64, device=W.device)
+    if order is None:
+        order = torch.empty(k, dtype=torch.int32, device=W.device)
+    _check(_lib().slim_salience_noalloc(_ptr(W), m, n, _ptr(h), group, _ptr(S), _ptr(order), _stream(stream)),
+           "slim_salience_noalloc")
     return S, order
 
 
