@@ -98,56 +98,137 @@ __host__ __device__ inline int blk_size(int64_t n, int b) {
 
 // ---------------------------------------------------------------- Cholesky pieces
 // Factor diagonal block K of A in place; write M_KK = L_KK^-1 into M.
+//
+// The pivots of a Cholesky factorization form a sequential chain (n of them
+// over the whole matrix), so each pivot step must be cheap. The 64 x 64 block
+// is processed in 16-wide sub-blocks:
+//   (1) warp 0 factors the 16 x 16 diagonal sub-block in shared memory (one
+//       rsqrt per pivot, warp-level synchronization only) and inverts it;
+//   (2) all warps compute the sub-panel below it, P = A_panel M_DD^T;
+//   (3) all warps apply the rank-16 update to the trailing lower triangle.
+// After the last sub-block, the off-diagonal 16 x 16 blocks of M = L^-1 come
+// from block forward substitution, M_IJ = -M_II sum_{K=J}^{I-1} L_IK M_KJ.
+constexpr int SB16 = 16;
 __global__ void __launch_bounds__(256) potrf_diag_kernel(double* __restrict__ A, double* __restrict__ M, int64_t n,
                                                          int K, DevStatus* st) {
   extern __shared__ double smem[];
   double (*s)[LDS] = reinterpret_cast<double (*)[LDS]>(smem);
-  double (*inv)[LDS] = reinterpret_cast<double (*)[LDS]>(smem + NB * LDS);
+  double (*mi)[LDS] = reinterpret_cast<double (*)[LDS]>(smem + NB * LDS);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nb = blk_size(n, K);
   const int64_t off = (int64_t)K * NB * n + (int64_t)K * NB;
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+  for (int e = tid; e < NB * NB; e += blockDim.x) {
     const int r = e / NB, c = e % NB;
     s[r][c] = (r < nb && c < nb && c <= r) ? A[off + (int64_t)r * n + c] : 0.0;
+    mi[r][c] = 0.0;
   }
   __syncthreads();
-  for (int j = 0; j < nb; ++j) {
-    if (threadIdx.x == 0) {
-      const double d = s[j][j];
-      if (!(d > 0.0)) {
-        record_failure(st, kStatusNotPD, K * NB + j);
-        s[j][j] = 1.0;
-      } else {
-        s[j][j] = sqrt(d);
+  for (int kb = 0; kb < nb; kb += SB16) {
+    const int w = (nb - kb < SB16) ? nb - kb : SB16;
+    if (warp == 0) {
+      // (1) unblocked Cholesky of the w x w diagonal sub-block
+      for (int p = 0; p < w; ++p) {
+        double d = s[kb + p][kb + p];
+        if (!(d > 0.0)) {
+          if (lane == 0) record_failure(st, kStatusNotPD, K * NB + kb + p);
+          d = 1.0;
+        }
+        const double ird = rsqrt(d);
+        __syncwarp();
+        if (lane > p && lane < w) s[kb + lane][kb + p] *= ird;
+        if (lane == p) s[kb + p][kb + p] = d * ird;
+        __syncwarp();
+#pragma unroll
+        for (int e = lane; e < SB16 * SB16; e += 32) {
+          const int i = e >> 4, l = e & 15;
+          if (i > p && i < w && l > p && l <= i)
+            s[kb + i][kb + l] = fma(-s[kb + i][kb + p], s[kb + l][kb + p], s[kb + i][kb + l]);
+        }
+        __syncwarp();
+      }
+      // inverse of the lower-triangular sub-block, one column per lane
+      if (lane < w) {
+        const int c = lane;
+        for (int i = c; i < w; ++i) {
+          double acc = (i == c) ? 1.0 : 0.0;
+          for (int l = c; l < i; ++l) acc = fma(-s[kb + i][kb + l], mi[kb + l][kb + c], acc);
+          mi[kb + i][kb + c] = acc / s[kb + i][kb + i];
+        }
       }
     }
     __syncthreads();
-    const double piv = s[j][j];
-    for (int i = j + 1 + threadIdx.x; i < nb; i += blockDim.x) s[i][j] = s[i][j] / piv;
-    __syncthreads();
-    const int rem = nb - j - 1;
-    for (int e = threadIdx.x; e < rem * rem; e += blockDim.x) {
-      const int i = j + 1 + e / rem, l = j + 1 + e % rem;
-      if (l <= i) s[i][l] = fma(-s[i][j], s[l][j], s[i][l]);
+    const int r0 = kb + w;
+    if (r0 < nb) {
+      // (2) sub-panel P[i][c] = sum_{l <= c} A[i][kb + l] M_DD[c][l], rows r0 .. nb-1
+      const int rows = nb - r0;
+      double pv[3];
+#pragma unroll
+      for (int q = 0; q < 3; ++q) {
+        const int e = tid + 256 * q;
+        pv[q] = 0.0;
+        if (e < rows * w) {
+          const int i = r0 + e / w, c = e % w;
+          double acc = 0.0;
+          for (int l = 0; l <= c; ++l) acc = fma(s[i][kb + l], mi[kb + c][kb + l], acc);
+          pv[q] = acc;
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int q = 0; q < 3; ++q) {
+        const int e = tid + 256 * q;
+        if (e < rows * w) s[r0 + e / w][kb + e % w] = pv[q];
+      }
+      __syncthreads();
+      // (3) trailing update of the lower triangle, rank w
+      for (int e = tid; e < rows * rows; e += blockDim.x) {
+        const int i = r0 + e / rows, l = r0 + e % rows;
+        if (l <= i) {
+          double acc = s[i][l];
+          for (int p = 0; p < w; ++p) acc = fma(-s[i][kb + p], s[l][kb + p], acc);
+          s[i][l] = acc;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // off-diagonal blocks of M by block forward substitution
+  const int nbl = (nb + SB16 - 1) / SB16;
+  for (int I = 1; I < nbl; ++I) {
+    const int i0 = I * SB16, wi = (nb - i0 < SB16) ? nb - i0 : SB16;
+    // T = sum_{K=J}^{I-1} L_IK M_KJ for every column block J < I, parked in mi[block I][0 .. i0)
+    for (int e = tid; e < wi * i0; e += blockDim.x) {
+      const int ii = e / i0, col = e % i0;
+      const int k0 = (col / SB16) * SB16;
+      double acc = 0.0;
+      for (int k = k0; k < i0; ++k) acc = fma(s[i0 + ii][k], mi[k][col], acc);
+      mi[i0 + ii][col] = acc;
     }
     __syncthreads();
-  }
-  // inverse of the lower-triangular block, one column per thread (forward substitution)
-  if (threadIdx.x < NB) {
-    const int c = threadIdx.x;
-    for (int i = 0; i < NB; ++i) inv[i][c] = 0.0;
-    if (c < nb) {
-      for (int i = c; i < nb; ++i) {
-        double acc = (i == c) ? 1.0 : 0.0;
-        for (int l = c; l < i; ++l) acc = fma(-s[i][l], inv[l][c], acc);
-        inv[i][c] = acc / s[i][i];
+    double tv[3];
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      const int e = tid + 256 * q;
+      tv[q] = 0.0;
+      if (e < wi * i0) {
+        const int ii = e / i0, col = e % i0;
+        double acc = 0.0;
+        for (int t = 0; t <= ii; ++t) acc = fma(mi[i0 + ii][i0 + t], mi[i0 + t][col], acc);
+        tv[q] = -acc;
       }
     }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      const int e = tid + 256 * q;
+      if (e < wi * i0) mi[i0 + e / i0][e % i0] = tv[q];
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < nb * nb; e += blockDim.x) {
+  for (int e = tid; e < nb * nb; e += blockDim.x) {
     const int r = e / nb, c = e % nb;
     A[off + (int64_t)r * n + c] = (c <= r) ? s[r][c] : 0.0;
-    M[off + (int64_t)r * n + c] = (c <= r) ? inv[r][c] : 0.0;
+    M[off + (int64_t)r * n + c] = (c <= r) ? mi[r][c] : 0.0;
   }
 }
 

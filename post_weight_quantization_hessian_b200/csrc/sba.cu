@@ -39,7 +39,7 @@
 //   x_to_f16       bf16 X -> fp16 (exact in fp16's normal range)
 //   x_split        fp32 X: X ~ X_hi + X_lo as two fp16 halves of X_cat
 //   sba_score      persistent tcgen05 kernel (below)
-//   sba_merge      per token: merges output-group partials in fp64 -> KL_t,
+//   sba_merge      per token: merges the output-tile partials in fp64 -> KL_t,
 //                  sums per token tile
 //   sba_final      KL_p = sum / N, p* = first argmin, bits
 #include <cstdint>
@@ -146,14 +146,16 @@ __global__ void x_split_kernel(const float* __restrict__ X, int64_t N, int64_t n
 
 // ---------------------------------------------------------------- scoring kernel
 constexpr int SB_BM = 128;        // tokens per tile (TMEM lanes)
-constexpr int SB_BN = 128;        // outputs per tile
-constexpr int SB_BK = 64;         // K elements per box (128 bytes of bf16)
+constexpr int SB_BN = 128;        // outputs per tile (one TMEM slot: y and d, 128 columns each)
+constexpr int SB_BK = 64;         // K elements per box (128 bytes of fp16)
 constexpr int SB_BOX = SB_BM * SB_BK * 2;  // 16 KB
 constexpr int SB_STAGE = 3 * SB_BOX;       // X, B1, B2
-constexpr int SB_GROUP_OUT = 2 * SB_BN;    // outputs per work unit (two TMEM slots)
 constexpr int SB_BAND = 32;                // token tiles per raster band
 constexpr int SB_MAX_K = 1024;
+constexpr int SB_EPI_WARPS = 8;            // two per TMEM lane quadrant, 64 columns each
+constexpr int SB_THREADS = 64 + 32 * SB_EPI_WARPS;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kC1 = kLog2e * kOpUnscale;  // exponent scale for accumulator (x 2^8) units
 
 struct SbaTmaps {
   CUtensorMap x, wb, e0, dp, dm;
@@ -162,10 +164,10 @@ struct SbaTmaps {
 struct SbaParams {
   int64_t N, m, n;
   int g, k, P, ksplit;
-  int n_tt, n_og, n_ot;   // token tiles, output groups, output tiles
-  int stages;
+  int n_tt, n_ot, stages;
+  int nA, nD;             // chunks of phase A and of one delta step
   const int32_t* order;
-  float* part;            // [n_tt][n_og][F][128], F = 2 + 2P
+  float* part;            // [n_tt][n_ot][F][128], F = 2 + 2P
   DevStatus* st;
 };
 
@@ -174,70 +176,114 @@ struct Chunk {
   int which;  // 0: phase A (Wb, E0); 1: Dp; 2: Dm
 };
 
-// Chunk list of item (p, s): returns the count; fills chunk c when idx == c.
-__device__ __forceinline__ int item_chunks(const SbaParams& p, const int32_t* order, int step, int idx, Chunk& ch) {
-  if (step == 0) {
-    const int kc_count = (int)((p.n + SB_BK - 1) / SB_BK);
-    const int cnt = kc_count * p.ksplit;
-    if (idx >= 0) {
-      const int kc = idx / p.ksplit, sx = idx - kc * p.ksplit;
-      ch.bcol = kc * SB_BK;
-      ch.xcol = ch.bcol + sx * (int)p.n;
-      ch.k16_lo = 0;
-      ch.k16_hi = 4;
-      ch.which = 0;
-    }
-    return cnt;
-  }
-  const int per_group = (p.g >= 64 ? p.g / 64 : 1) * p.ksplit;
-  const int cnt = 2 * per_group;
-  if (idx >= 0) {
-    const int gi = idx / per_group, rem = idx - gi * per_group;
-    const int c = gi == 0 ? order[step - 1] : order[p.k - step];
-    const int bx = rem / p.ksplit, sx = rem - bx * p.ksplit;
-    if (p.g >= 64) {
-      ch.bcol = c * p.g + 64 * bx;
-      ch.k16_lo = 0;
-      ch.k16_hi = 4;
-    } else {
-      const int col = c * p.g;
-      ch.bcol = (col / 64) * 64;
-      ch.k16_lo = (col % 64) / 16;
-      ch.k16_hi = ch.k16_lo + p.g / 16;
-    }
-    ch.xcol = ch.bcol + sx * (int)p.n;
-    ch.which = gi == 0 ? 1 : 2;
-  }
-  return cnt;
-}
-
-__device__ __forceinline__ void unit_decode(const SbaParams& p, int u, int& tt, int& og) {
-  const int band_start = (u / (SB_BAND * p.n_og)) * SB_BAND;
+// Work tile u -> (token tile, output tile), raster bands of SB_BAND token tiles.
+__device__ __forceinline__ void tile_decode(const SbaParams& p, int u, int& tt, int& ot) {
+  const int band_start = (u / (SB_BAND * p.n_ot)) * SB_BAND;
   const int bc = (p.n_tt - band_start < SB_BAND) ? p.n_tt - band_start : SB_BAND;
-  const int r = u - band_start * p.n_og;
-  og = r / bc;
-  tt = band_start + (r - og * bc);
+  const int r = u - band_start * p.n_ot;
+  ot = r / bc;
+  tt = band_start + (r - ot * bc);
 }
 
-__global__ void __launch_bounds__(192, 1) sba_score_kernel(const __grid_constant__ SbaTmaps tm, SbaParams p) {
+// The MMA issue order of one CTA's T tiles, shared by the TMA producer and the
+// MMA issuer. Tile i alternates between the two TMEM slots. Phase A of tile i
+// is cut into slices placed before each delta step of tile i-1, so the tensor
+// pipe keeps busy while the epilogue digests tile i-1's candidates:
+//   A(T0) | A(T1) slice, D1(T0), A(T1) slice, D2(T0), ... | A(T2) slice, D1(T1), ... | ..., D_{P-1}(T_last)
+// f(tile, step, chunk_begin, chunk_end, item_chunks) is called once per slice
+// of an item (step 0: phase A, nA chunks; step p: delta p, nD chunks); it
+// returns false to abort the walk.
+template <class F>
+__device__ __forceinline__ bool walk_schedule(const SbaParams& p, int T, F&& f) {
+  const int steps = p.P - 1;
+  for (int i = 0; i <= T; ++i) {
+    const bool hasA = i < T, hasD = i > 0 && steps > 0;
+    if (!hasD) {
+      if (hasA && !f(i, 0, 0, p.nA, p.nA)) return false;
+      continue;
+    }
+    int a_done = 0;
+    for (int s = 1; s <= steps; ++s) {
+      if (hasA) {
+        const int a_to = (int)((int64_t)s * p.nA / steps);
+        if (a_to > a_done && !f(i, 0, a_done, a_to, p.nA)) return false;
+        a_done = a_to;
+      }
+      if (!f(i - 1, s, 0, p.nD, p.nD)) return false;
+    }
+  }
+  return true;
+}
+
+// Per-item chunk geometry without divisions in the chunk loop. Phase A chunk
+// c: K box c >> (ksplit - 1), X half c & (ksplit - 1). Delta chunk c: group
+// c / per_group (promoted first), then K box and X half within the group.
+struct ItemGeom {
+  int step, ks_shift, per_group, col_up, col_dn, k16_lo_up, k16_lo_dn, k16_n;
+};
+__device__ __forceinline__ ItemGeom item_geom(const SbaParams& p, const int32_t* order, int step) {
+  ItemGeom g;
+  g.step = step;
+  g.ks_shift = p.ksplit == 2 ? 1 : 0;
+  g.per_group = p.nD >> 1;
+  g.k16_n = p.g >= 64 ? 4 : p.g / 16;
+  g.col_up = g.col_dn = 0;
+  g.k16_lo_up = g.k16_lo_dn = 0;
+  if (step > 0) {
+    const int cu = order[step - 1] * p.g, cd = order[p.k - step] * p.g;
+    g.col_up = p.g >= 64 ? cu : (cu & ~63);
+    g.col_dn = p.g >= 64 ? cd : (cd & ~63);
+    g.k16_lo_up = p.g >= 64 ? 0 : (cu & 63) >> 4;
+    g.k16_lo_dn = p.g >= 64 ? 0 : (cd & 63) >> 4;
+  }
+  return g;
+}
+__device__ __forceinline__ void chunk_at(const SbaParams& p, const ItemGeom& g, int c, Chunk& ch) {
+  const int sx = c & ((1 << g.ks_shift) - 1);
+  if (g.step == 0) {
+    ch.bcol = (c >> g.ks_shift) * SB_BK;
+    ch.k16_lo = 0;
+    ch.k16_hi = 4;
+    ch.which = 0;
+  } else {
+    const bool up = c < g.per_group;
+    const int rem = up ? c : c - g.per_group;
+    ch.bcol = (up ? g.col_up : g.col_dn) + (rem >> g.ks_shift) * SB_BK;
+    ch.k16_lo = up ? g.k16_lo_up : g.k16_lo_dn;
+    ch.k16_hi = ch.k16_lo + g.k16_n;
+    ch.which = up ? 1 : 2;
+  }
+  ch.xcol = ch.bcol + (sx ? (int)p.n : 0);
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_constant__ SbaTmaps tm, SbaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * SB_STAGE);
   uint64_t* empty = full + S;
-  uint64_t* afull = empty + S;   // [2]
-  uint64_t* afree = afull + 2;   // [2]
+  uint64_t* afull = empty + S;   // [2] item accumulated in TMEM slot s
+  uint64_t* afree = afull + 2;   // [2] epilogue done with slot s's last item
   uint64_t* done = afree + 2;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* xbar = done + 1;     // [4] column-half exchange, one per TMEM lane quadrant (64 threads)
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(xbar + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-  int32_t* s_order = reinterpret_cast<int32_t*>(tslot + 2);
+  float* xbuf = reinterpret_cast<float*>(tslot + 2);            // [2][4][2][3][32] half-to-half exchange
+  int32_t* s_order = reinterpret_cast<int32_t*>(xbuf + 2 * 4 * 2 * 3 * 32);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int c = threadIdx.x; c < p.k; c += blockDim.x) s_order[c] = p.order[c];
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&afull[s], 1); mbar_init(&afree[s], 4); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&afull[s], 1); mbar_init(&afree[s], SB_EPI_WARPS); }
     mbar_init(done, 1);
+    for (int qq = 0; qq < 4; ++qq) mbar_init(&xbar[qq], 64);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -245,37 +291,58 @@ __global__ void __launch_bounds__(192, 1) sba_score_kernel(const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tslot;
-  const int units = p.n_tt * p.n_og;
+  const int tiles = p.n_tt * p.n_ot;
+  const int T = (tiles > (int)blockIdx.x) ? (tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
-      const void* bmaps[3][2] = {{&tm.wb, &tm.e0}, {&tm.dp, nullptr}, {&tm.dm, nullptr}};
-      uint32_t it = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        int tt, og;
-        unit_decode(p, u, tt, og);
-        const int nslots = (p.n_ot - 2 * og) < 2 ? (p.n_ot - 2 * og) : 2;
-        for (int step = 0; step < p.P && ok; ++step)
-          for (int s = 0; s < nslots && ok; ++s) {
+      uint32_t it = 0;      // chunks issued (for the final drain)
+      int st = 0;           // stage ring position and its phase bit
+      uint32_t ph = 0;
+      walk_schedule(p, T, [&](int ti, int step, int c0, int c1, int) -> bool {
+        int tt, ot;
+        tile_decode(p, (int)blockIdx.x + ti * (int)gridDim.x, tt, ot);
+        const ItemGeom geo = item_geom(p, s_order, step);
+        const int brow = ot * SB_BN, xrow = tt * SB_BM;
+        for (int c = c0; c < c1; ++c) {
+          Chunk ch;
+          chunk_at(p, geo, c, ch);
+          if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, p.st, 200 + st)) return false;
+          uint8_t* sb = smem + st * SB_STAGE;
+          mbar_arrive_expect_tx(&full[st], (ch.which == 0 ? 3 : 2) * SB_BOX);
+          tma_load_2d(sb, &tm.x, &full[st], ch.xcol, xrow);
+          if (ch.which == 0) {
+            tma_load_2d(sb + SB_BOX, &tm.wb, &full[st], ch.bcol, brow);
+            tma_load_2d(sb + 2 * SB_BOX, &tm.e0, &full[st], ch.bcol, brow);
+          } else {
+            tma_load_2d(sb + SB_BOX, ch.which == 1 ? (const void*)&tm.dp : (const void*)&tm.dm, &full[st], ch.bcol,
+                        brow);
+          }
+          ++it;
+          if (++st == S) { st = 0; ph ^= 1; }
+        }
+        // warm L2 with what this tile needs next: the following phase-A slice, or the next delta step
+        auto prefetch = [&](const ItemGeom& g, int a, int b) {
+          for (int c = a; c < b; ++c) {
             Chunk ch;
-            const int nch = item_chunks(p, s_order, step, -1, ch);
-            const int brow = (og * 2 + s) * SB_BN;
-            for (int ci = 0; ci < nch; ++ci, ++it) {
-              item_chunks(p, s_order, step, ci, ch);
-              const int st = it % S;
-              const uint32_t ph = (it / S) & 1;
-              if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, p.st, 200 + st)) { ok = false; break; }
-              uint8_t* sb = smem + st * SB_STAGE;
-              const int nbox = ch.which == 0 ? 3 : 2;
-              mbar_arrive_expect_tx(&full[st], nbox * SB_BOX);
-              tma_load_2d(sb, &tm.x, &full[st], ch.xcol, tt * SB_BM);
-              tma_load_2d(sb + SB_BOX, bmaps[ch.which][0], &full[st], ch.bcol, brow);
-              if (ch.which == 0) tma_load_2d(sb + 2 * SB_BOX, bmaps[0][1], &full[st], ch.bcol, brow);
+            chunk_at(p, g, c, ch);
+            tma_prefetch_l2(&tm.x, ch.xcol, xrow);
+            if (ch.which == 0) {
+              tma_prefetch_l2(&tm.wb, ch.bcol, brow);
+              tma_prefetch_l2(&tm.e0, ch.bcol, brow);
+            } else {
+              tma_prefetch_l2(ch.which == 1 ? (const void*)&tm.dp : (const void*)&tm.dm, ch.bcol, brow);
             }
           }
-      }
+        };
+        if (step == 0) {
+          prefetch(geo, c1, min(p.nA, c1 + (c1 - c0)));
+        } else if (step + 1 < p.P) {
+          prefetch(item_geom(p, s_order, step + 1), 0, p.nD);
+        }
+        return true;
+      });
       // let every issued copy land before the CTA can exit
       for (uint32_t j = (it > (uint32_t)S ? it - S : 0); j < it; ++j) {
         uint64_t t0 = global_ns();
@@ -286,141 +353,167 @@ __global__ void __launch_bounds__(192, 1) sba_score_kernel(const __grid_constant
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(SB_BM, SB_BN, false, false);
-      uint32_t it = 0;
+      constexpr uint32_t idesc2 = idesc_f16_f32(SB_BM, 2 * SB_BN, false, false);
+      int st = 0;
+      uint32_t ph = 0;
       uint32_t cnt[2] = {0, 0};
-      bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        int tt, og;
-        unit_decode(p, u, tt, og);
-        const int nslots = (p.n_ot - 2 * og) < 2 ? (p.n_ot - 2 * og) : 2;
-        for (int step = 0; step < p.P && ok; ++step)
-          for (int s = 0; s < nslots && ok; ++s) {
-            if (!mbar_wait(&afree[s], (cnt[s] & 1) ^ 1, abort_flag, p.st, 220 + s)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t ty = tbase + s * 256, td = ty + 128;
-            Chunk ch;
-            const int nch = item_chunks(p, s_order, step, -1, ch);
-            for (int ci = 0; ci < nch; ++ci, ++it) {
-              item_chunks(p, s_order, step, ci, ch);
-              const int st = it % S;
-              const uint32_t ph = (it / S) & 1;
-              if (!mbar_wait(&full[st], ph, abort_flag, p.st, 230 + st)) { ok = false; break; }
-              tc_fence_after();
-              const uint32_t xa = smem_u32(smem + st * SB_STAGE);
-              for (int k16 = ch.k16_lo; k16 < ch.k16_hi; ++k16) {
-                const uint64_t ad = sdesc_sw128(xa + k16 * 32, 16, 1024);
-                const uint64_t b1 = sdesc_sw128(xa + SB_BOX + k16 * 32, 16, 1024);
-                if (ch.which == 0) {
-                  const uint32_t acc = (ci > 0 || k16 > ch.k16_lo) ? 1u : 0u;
-                  const uint64_t b2 = sdesc_sw128(xa + 2 * SB_BOX + k16 * 32, 16, 1024);
-                  tc_mma_f16(ty, ad, b1, idesc, acc);
-                  tc_mma_f16(td, ad, b2, idesc, acc);
-                } else {
-                  tc_mma_f16(td, ad, b1, idesc, 1u);
-                }
-              }
-              tc_commit(&empty[st]);
+      walk_schedule(p, T, [&](int ti, int step, int c0, int c1, int nitem) -> bool {
+        const int slot = ti & 1;
+        if (c0 == 0) {
+          if (!mbar_wait(&afree[slot], (cnt[slot] & 1) ^ 1, abort_flag, p.st, 220 + slot)) return false;
+          tc_fence_after();
+        }
+        const ItemGeom geo = item_geom(p, s_order, step);
+        const uint32_t ty = tbase + slot * 256, td = ty + 128;
+        for (int c = c0; c < c1; ++c) {
+          Chunk ch;
+          chunk_at(p, geo, c, ch);
+          if (!mbar_wait(&full[st], ph, abort_flag, p.st, 230 + st)) return false;
+          tc_fence_after();
+          const uint32_t xa = smem_u32(smem + st * SB_STAGE);
+          const uint64_t ad0 = sdesc_sw128(xa, 16, 1024);
+          const uint64_t b10 = sdesc_sw128(xa + SB_BOX, 16, 1024);
+          if (ch.which == 0) {
+            // the Wb and E0 boxes are adjacent (256 B-operand rows), and so are y and d in TMEM:
+            // one N = 256 MMA per k16 step writes both accumulators
+#pragma unroll
+            for (int k16 = 0; k16 < 4; ++k16) {
+              const uint32_t acc = (c > 0 || k16 > 0) ? 1u : 0u;
+              // advancing 32 bytes along K = +2 in the descriptor's 16-byte start-address field
+              tc_mma_f16(ty, ad0 + 2 * k16, b10 + 2 * k16, idesc2, acc);
             }
-            if (!ok) break;
-            tc_commit(&afull[s]);
-            ++cnt[s];
+          } else {
+            for (int k16 = ch.k16_lo; k16 < ch.k16_hi; ++k16)
+              tc_mma_f16(td, ad0 + 2 * k16, b10 + 2 * k16, idesc, 1u);
           }
-      }
+          tc_commit(&empty[st]);
+          if (++st == S) { st = 0; ph ^= 1; }
+        }
+        if (c1 == nitem) {
+          tc_commit(&afull[slot]);
+          ++cnt[slot];
+        }
+        return true;
+      });
       tc_commit(done);
       uint64_t t0 = global_ns();
       while (!mbar_try_wait(done, 0) && global_ns() - t0 < kWaitLimitNs) {}
     }
   } else {
-    // ------------------------------------------------ epilogue: 4 warps, one token row per thread
-    const int wq = warp & 3;
-    const int r = wq * 32 + lane;
+    // ------------------------------------------------ epilogue: 8 warps, token row per lane, 64 columns per warp
+    const int q = warp & 3;                 // TMEM lane quadrant this warp may access
+    const int hf = (warp - 2) >> 2;         // which 64 of the tile's 128 columns
+    const int r = q * 32 + lane;            // token row inside the tile
     const int F = 2 + 2 * p.P;
-    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     uint32_t cnt[2] = {0, 0};
+    int xc = 0;                             // exchange counter (double-buffered xbuf)
+    auto xb = [&](int buf, int half, int val) -> float& { return xbuf[((((buf * 4) + q) * 2 + half) * 3 + val) * 32 + lane]; };
+    // both 32-lane halves of quadrant q arrive, then wait (bounded) for exchange xc's phase
+    auto xsync = [&]() -> bool {
+      mbar_arrive(&xbar[q]);
+      return mbar_wait(&xbar[q], xc & 1, abort_flag, p.st, 250 + q);
+    };
     bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-      int tt, og;
-      unit_decode(p, u, tt, og);
-      const int nslots = (p.n_ot - 2 * og) < 2 ? (p.n_ot - 2 * og) : 2;
-      float* outp = p.part + ((size_t)tt * p.n_og + og) * F * SB_BM + r;
-      float Ms[2] = {0.f, 0.f}, Sys[2] = {0.f, 0.f}, fs[2] = {1.f, 1.f};
-      float sq_s0 = 0.f, a_s0 = 0.f;
-      for (int step = 0; step < p.P && ok; ++step)
-        for (int s = 0; s < nslots && ok; ++s) {
-          if (!mbar_wait(&afull[s], cnt[s] & 1, abort_flag, p.st, 240 + s)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t ty = tbase + lane_off + s * 256, td = ty + 128;
-          const int64_t col0 = (int64_t)(og * 2 + s) * SB_BN;
-          float sq = 0.f, a = 0.f;
-          if (step == 0) {
-            float mx = -3.0e38f;
+    for (int ti = 0; ti < T && ok; ++ti) {
+      const int slot = ti & 1;
+      int tt, ot;
+      tile_decode(p, (int)blockIdx.x + ti * (int)gridDim.x, tt, ot);
+      const int64_t col0 = (int64_t)ot * SB_BN + hf * 64;
+      const int nvalid = (int)((p.m - col0) < 0 ? 0 : ((p.m - col0) > 64 ? 64 : (p.m - col0)));
+      float* outp = p.part + ((size_t)tt * p.n_ot + ot) * F * SB_BM + r;
+      const uint32_t ty = tbase + lane_off + slot * 256 + hf * 64, td = ty + 128;
+      float Mt = 0.f, syt = 0.f;
+      for (int step = 0; step < p.P; ++step) {
+        if (!mbar_wait(&afull[slot], cnt[slot] & 1, abort_flag, p.st, 240 + slot)) { ok = false; break; }
+        tc_fence_after();
+        float sq0 = 0.f, sq1 = 0.f, a0 = 0.f, a1 = 0.f, sy0 = 0.f, sy1 = 0.f;
+        if (step == 0) {
+          float mx = -3.0e38f;
 #pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
-              uint32_t yv[32];
-              tmem_ld32(ty + cc * 32, yv);
-              tc_wait_ld();
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t yv[32];
+            tmem_ld32(ty + cc * 32, yv);
+            tc_wait_ld();
 #pragma unroll
-              for (int v = 0; v < 32; ++v)
-                if (col0 + cc * 32 + v < p.m) mx = fmaxf(mx, __uint_as_float(yv[v]) * kOpUnscale);
-            }
-            float sy = 0.f;
-#pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
-              uint32_t yv[32], dv[32];
-              tmem_ld32(ty + cc * 32, yv);
-              tmem_ld32(td + cc * 32, dv);
-              tc_wait_ld();
-#pragma unroll
-              for (int v = 0; v < 32; ++v) {
-                const bool valid = col0 + cc * 32 + v < p.m;
-                const float y = __uint_as_float(yv[v]) * kOpUnscale;
-                const float d = __uint_as_float(dv[v]) * kOpUnscale;
-                const float ey = valid ? exp2f((y - mx) * kLog2e) : 0.f;
-                sy += ey;
-                sq = fmaf(ey, exp2f(d * kLog2e), sq);
-                a = fmaf(ey, d, a);
-                yv[v] = __float_as_uint(ey);
-              }
-              tmem_st32(ty + cc * 32, yv);
-            }
-            tc_wait_st();
-            Ms[s] = mx;
-            Sys[s] = sy;
-          } else {
-#pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
-              uint32_t ev[32], dv[32];
-              tmem_ld32(ty + cc * 32, ev);
-              tmem_ld32(td + cc * 32, dv);
-              tc_wait_ld();
-#pragma unroll
-              for (int v = 0; v < 32; ++v) {
-                const float ey = __uint_as_float(ev[v]);
-                const float d = __uint_as_float(dv[v]) * kOpUnscale;
-                sq = fmaf(ey, exp2f(d * kLog2e), sq);
-                a = fmaf(ey, d, a);
-              }
-            }
+            for (int v = 0; v < 32; ++v)
+              if (cc * 32 + v < nvalid) mx = fmaxf(mx, __uint_as_float(yv[v]));
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&afree[s]);
-          ++cnt[s];
-          if (s == 0) { sq_s0 = sq; a_s0 = a; }
-          if (s == nslots - 1) {
-            if (step == 0) {
-              const float M = nslots == 2 ? fmaxf(Ms[0], Ms[1]) : Ms[0];
-              fs[0] = exp2f((Ms[0] - M) * kLog2e);
-              fs[1] = nslots == 2 ? exp2f((Ms[1] - M) * kLog2e) : 0.f;
-              outp[0] = M;
-              outp[SB_BM] = Sys[0] * fs[0] + (nslots == 2 ? Sys[1] * fs[1] : 0.f);
+          // tile maximum: combine with the partner warp holding the other 64 columns
+          xb(xc & 1, hf, 0) = mx;
+          if (!xsync()) { ok = false; break; }
+          mx = fmaxf(mx, xb(xc & 1, hf ^ 1, 0));
+          ++xc;
+          const float mb = -mx * kC1;
+#pragma unroll 1
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t yv[32], dv[32];
+            tmem_ld32(ty + cc * 32, yv);
+            tmem_ld32(td + cc * 32, dv);
+            tc_wait_ld();
+#pragma unroll
+            for (int v = 0; v < 32; v += 2) {
+              const bool ok0 = cc * 32 + v < nvalid, ok1 = cc * 32 + v + 1 < nvalid;
+              const float ey0 = ok0 ? ex2(fmaf(__uint_as_float(yv[v]), kC1, mb)) : 0.f;
+              const float ey1 = ok1 ? ex2(fmaf(__uint_as_float(yv[v + 1]), kC1, mb)) : 0.f;
+              const float d0 = __uint_as_float(dv[v]), d1 = __uint_as_float(dv[v + 1]);
+              sy0 += ey0;
+              sy1 += ey1;
+              sq0 = fmaf(ey0, ex2(d0 * kC1), sq0);
+              sq1 = fmaf(ey1, ex2(d1 * kC1), sq1);
+              a0 = fmaf(ey0, d0, a0);
+              a1 = fmaf(ey1, d1, a1);
+              yv[v] = __float_as_uint(ey0);
+              yv[v + 1] = __float_as_uint(ey1);
             }
-            float sqt = sq_s0 * fs[0], at = a_s0 * fs[0];
-            if (nslots == 2) { sqt = fmaf(sq, fs[1], sqt); at = fmaf(a, fs[1], at); }
-            outp[(size_t)(2 + 2 * step) * SB_BM] = sqt;
-            outp[(size_t)(3 + 2 * step) * SB_BM] = at;
+            tmem_st32(ty + cc * 32, yv);
+          }
+          tc_wait_st();
+          Mt = mx;
+        } else {
+#pragma unroll 1
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t ev[32], dv[32];
+            tmem_ld32(ty + cc * 32, ev);
+            tmem_ld32(td + cc * 32, dv);
+            tc_wait_ld();
+#pragma unroll
+            for (int v = 0; v < 32; v += 2) {
+              const float ey0 = __uint_as_float(ev[v]), ey1 = __uint_as_float(ev[v + 1]);
+              const float d0 = __uint_as_float(dv[v]), d1 = __uint_as_float(dv[v + 1]);
+              sq0 = fmaf(ey0, ex2(d0 * kC1), sq0);
+              sq1 = fmaf(ey1, ex2(d1 * kC1), sq1);
+              a0 = fmaf(ey0, d0, a0);
+              a1 = fmaf(ey1, d1, a1);
+            }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afree[slot]);
+        ++cnt[slot];
+        // combine the two column halves; half 0 writes this tile's partial statistics
+        float sy = sy0 + sy1, sq = sq0 + sq1, a = a0 + a1;
+        if (hf == 1) {
+          xb(xc & 1, 1, 0) = sy;
+          xb(xc & 1, 1, 1) = sq;
+          xb(xc & 1, 1, 2) = a;
+        }
+        if (!xsync()) { ok = false; break; }
+        if (hf == 0) {
+          sy += xb(xc & 1, 1, 0);
+          sq += xb(xc & 1, 1, 1);
+          a += xb(xc & 1, 1, 2);
+          if (step == 0) {
+            syt = sy;
+            outp[0] = Mt * kOpUnscale;
+            outp[SB_BM] = syt;
+          }
+          outp[(size_t)(2 + 2 * step) * SB_BM] = sq;
+          outp[(size_t)(3 + 2 * step) * SB_BM] = a * kOpUnscale;
+        }
+        ++xc;
+      }
     }
   }
   __syncthreads();
@@ -431,25 +524,25 @@ __global__ void __launch_bounds__(192, 1) sba_score_kernel(const __grid_constant
 }
 
 // ---------------------------------------------------------------- merge and final
-__global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict__ part, int n_og, int P, int64_t N,
+__global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict__ part, int n_ot, int P, int64_t N,
                                                         int n_tt, double* __restrict__ kl_part) {
-  extern __shared__ float s_f[];  // [n_og][128] scale factors
+  extern __shared__ float s_f[];  // [n_ot][128] scale factors (one partial set per output tile)
   __shared__ double red[4];
   const int tt = blockIdx.x, r = threadIdx.x;
   const int F = 2 + 2 * P;
   const bool valid = (int64_t)tt * SB_BM + r < N;
-  const float* base = part + (size_t)tt * n_og * F * SB_BM + r;
+  const float* base = part + (size_t)tt * n_ot * F * SB_BM + r;
   float M = -3.0e38f;
-  for (int og = 0; og < n_og; ++og) M = fmaxf(M, base[(size_t)og * F * SB_BM]);
+  for (int og = 0; og < n_ot; ++og) M = fmaxf(M, base[(size_t)og * F * SB_BM]);
   double Sy = 0.0;
-  for (int og = 0; og < n_og; ++og) {
+  for (int og = 0; og < n_ot; ++og) {
     const float f = exp2f((base[(size_t)og * F * SB_BM] - M) * kLog2e);
     s_f[og * SB_BM + r] = f;
     Sy += (double)base[(size_t)og * F * SB_BM + SB_BM] * (double)f;
   }
   for (int q = 0; q < P; ++q) {
     double sq = 0.0, a = 0.0;
-    for (int og = 0; og < n_og; ++og) {
+    for (int og = 0; og < n_ot; ++og) {
       const double f = s_f[og * SB_BM + r];
       sq += (double)base[((size_t)og * F + 2 + 2 * q) * SB_BM] * f;
       a += (double)base[((size_t)og * F + 3 + 2 * q) * SB_BM] * f;
@@ -494,7 +587,7 @@ __global__ void sba_final_kernel(const double* __restrict__ kl_part, int n_tt, i
 
 // ---------------------------------------------------------------- host side
 struct SbaPlan {
-  int k, P, ksplit, n_tt, n_og, n_ot, stages;
+  int k, P, ksplit, n_tt, n_ot, stages, nA, nD;
   size_t off_wb, off_e0, off_dp, off_dm, off_xc, off_part, off_klp, total;
   size_t smem;
 };
@@ -508,7 +601,8 @@ SbaPlan sba_plan(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
   pl.ksplit = xdtype == 1 ? 1 : 2;
   pl.n_tt = (int)((N + SB_BM - 1) / SB_BM);
   pl.n_ot = (int)((m + SB_BN - 1) / SB_BN);
-  pl.n_og = (pl.n_ot + 1) / 2;
+  pl.nA = (int)((n + SB_BK - 1) / SB_BK) * pl.ksplit;
+  pl.nD = 2 * (group >= 64 ? group / 64 : 1) * pl.ksplit;
   const size_t wbytes = (size_t)m * n * 2;
   size_t off = 0;
   pl.off_wb = off; off = align256(off + wbytes);
@@ -516,10 +610,10 @@ SbaPlan sba_plan(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
   pl.off_dp = off; off = align256(off + wbytes);
   pl.off_dm = off; off = align256(off + wbytes);
   pl.off_xc = off; off = align256(off + (size_t)N * pl.ksplit * n * 2);
-  pl.off_part = off; off = align256(off + (size_t)pl.n_tt * pl.n_og * (2 + 2 * pl.P) * SB_BM * sizeof(float));
+  pl.off_part = off; off = align256(off + (size_t)pl.n_tt * pl.n_ot * (2 + 2 * pl.P) * SB_BM * sizeof(float));
   pl.off_klp = off; off = align256(off + (size_t)pl.P * pl.n_tt * sizeof(double));
   pl.total = off;
-  const size_t fixed = 1024 + 256 + (size_t)pl.k * 4 + 64;
+  const size_t fixed = 1024 + 512 + 2 * 4 * 2 * 3 * 32 * sizeof(float) + (size_t)pl.k * 4 + 64;
   int st = 4;
   while (st > 2 && fixed + (size_t)st * SB_STAGE > 227 * 1024) --st;
   pl.stages = st;
@@ -572,21 +666,21 @@ cudaError_t launch_sba(const float* W, int64_t m, int64_t n, const void* X, int 
 
   SbaParams p;
   p.N = N; p.m = m; p.n = n; p.g = group; p.k = pl.k; p.P = pl.P; p.ksplit = pl.ksplit;
-  p.n_tt = pl.n_tt; p.n_og = pl.n_og; p.n_ot = pl.n_ot; p.stages = pl.stages;
+  p.n_tt = pl.n_tt; p.n_ot = pl.n_ot; p.stages = pl.stages; p.nA = pl.nA; p.nD = pl.nD;
   p.order = order; p.part = part; p.st = st;
   cudaError_t e = cudaFuncSetAttribute(sba_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
   if (e != cudaSuccess) return e;
-  const int units = pl.n_tt * pl.n_og;
-  const int grid = units < num_sms ? units : num_sms;
+  const int tiles = pl.n_tt * pl.n_ot;
+  const int grid = tiles < num_sms ? tiles : num_sms;
   if (kev) cudaEventRecord(kev[0], s);
-  sba_score_kernel<<<grid, 192, pl.smem, s>>>(tm, p);
+  sba_score_kernel<<<grid, SB_THREADS, pl.smem, s>>>(tm, p);
   if (kev) cudaEventRecord(kev[1], s);
-  const size_t msmem = (size_t)pl.n_og * SB_BM * sizeof(float);
+  const size_t msmem = (size_t)pl.n_ot * SB_BM * sizeof(float);
   if (msmem > 48 * 1024) {
     e = cudaFuncSetAttribute(sba_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
     if (e != cudaSuccess) return e;
   }
-  sba_merge_kernel<<<pl.n_tt, SB_BM, msmem, s>>>(part, pl.n_og, pl.P, N, pl.n_tt, klp);
+  sba_merge_kernel<<<pl.n_tt, SB_BM, msmem, s>>>(part, pl.n_ot, pl.P, N, pl.n_tt, klp);
   sba_final_kernel<<<1, 256, 0, s>>>(klp, pl.n_tt, pl.P, N, order, pl.k, avg_bits, kl, p_star, bits);
   count_launches(5);
   return cudaGetLastError();
