@@ -14,10 +14,12 @@
 //     rowmult      M_IJ = M_II R_IJ for J < I (R accumulates -sum L_IK M_KJ)
 //     update       R_I'J -= L_I'I M_IJ for I' > I, J <= I
 //   Column norms   h_j = sum_{i >= j} M_ij^2 (partials, then a fixed-order sum)
+// The inverse steps run on a side stream, overlapping the Cholesky chain.
 //
 // Flops are n^3/3 for each half. A non-positive pivot records SLIM_ENOTPD with
 // its index; the remaining kernels run to completion on the bad values.
 #include <cstdint>
+#include <vector>
 #include "common.cuh"
 
 namespace slim {
@@ -103,7 +105,9 @@ __host__ __device__ inline int blk_size(int64_t n, int b) {
 // over the whole matrix), so each pivot step must be cheap. The 64 x 64 block
 // is processed in 16-wide sub-blocks:
 //   (1) warp 0 factors the 16 x 16 diagonal sub-block in shared memory (one
-//       rsqrt per pivot, warp-level synchronization only) and inverts it;
+//       rsqrt per pivot, warp-level synchronization only) and, in the same
+//       pivot loop, inverts it (right-looking: row p of M is row p of R
+//       scaled by 1/L_pp, then R_ic -= L_ip M_pc for i > p, c <= p);
 //   (2) all warps compute the sub-panel below it, P = A_panel M_DD^T;
 //   (3) all warps apply the rank-16 update to the trailing lower triangle.
 // After the last sub-block, the off-diagonal 16 x 16 blocks of M = L^-1 come
@@ -120,40 +124,55 @@ __global__ void __launch_bounds__(256) potrf_diag_kernel(double* __restrict__ A,
   for (int e = tid; e < NB * NB; e += blockDim.x) {
     const int r = e / NB, c = e % NB;
     s[r][c] = (r < nb && c < nb && c <= r) ? A[off + (int64_t)r * n + c] : 0.0;
-    mi[r][c] = 0.0;
+    mi[r][c] = (r == c) ? 1.0 : 0.0;
   }
   __syncthreads();
   for (int kb = 0; kb < nb; kb += SB16) {
     const int w = (nb - kb < SB16) ? nb - kb : SB16;
     if (warp == 0) {
-      // (1) unblocked Cholesky of the w x w diagonal sub-block
-      for (int p = 0; p < w; ++p) {
-        double d = s[kb + p][kb + p];
+      // (1) unblocked Cholesky of the 16 x 16 diagonal sub-block, and its inverse, in
+      // registers: lane = row i (lane & 15), columns 8h .. 8h+7 (h = lane >> 4). Each
+      // pivot's column and row travel by shuffles; the loop is unrolled so register
+      // slots are static. (n is a multiple of 32, so sub-blocks are always 16 wide.)
+      const int i = lane & 15, h = lane >> 4;
+      double a[8], r[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        a[c] = s[kb + i][kb + 8 * h + c];
+        r[c] = (i == 8 * h + c) ? 1.0 : 0.0;
+      }
+#pragma unroll
+      for (int p = 0; p < SB16; ++p) {
+        const int ph = p >> 3, pc = p & 7;
+        double d = __shfl_sync(0xffffffffu, a[pc], p + 16 * ph);
         if (!(d > 0.0)) {
           if (lane == 0) record_failure(st, kStatusNotPD, K * NB + kb + p);
           d = 1.0;
         }
         const double ird = rsqrt(d);
-        __syncwarp();
-        if (lane > p && lane < w) s[kb + lane][kb + p] *= ird;
-        if (lane == p) s[kb + p][kb + p] = d * ird;
-        __syncwarp();
+        const double ci = __shfl_sync(0xffffffffu, a[pc], i + 16 * ph);   // unscaled a_ip
+        const double fi = ci * ird;                                        // L_ip
+        double cl[8], rp[8];
 #pragma unroll
-        for (int e = lane; e < SB16 * SB16; e += 32) {
-          const int i = e >> 4, l = e & 15;
-          if (i > p && i < w && l > p && l <= i)
-            s[kb + i][kb + l] = fma(-s[kb + i][kb + p], s[kb + l][kb + p], s[kb + i][kb + l]);
+        for (int c = 0; c < 8; ++c) {
+          cl[c] = __shfl_sync(0xffffffffu, a[pc], 8 * h + c + 16 * ph) * ird;   // L_lp
+          rp[c] = __shfl_sync(0xffffffffu, r[c], p + 16 * h) * ird;             // M_pl
         }
-        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int l = 8 * h + c;
+          if (l == p) a[c] = (i == p) ? d * ird : ((i > p) ? fi : a[c]);
+          else if (l > p && l <= i) a[c] = fma(-fi, cl[c], a[c]);
+          if (l <= p) {
+            if (i == p) r[c] *= ird;
+            else if (i > p) r[c] = fma(-fi, rp[c], r[c]);
+          }
+        }
       }
-      // inverse of the lower-triangular sub-block, one column per lane
-      if (lane < w) {
-        const int c = lane;
-        for (int i = c; i < w; ++i) {
-          double acc = (i == c) ? 1.0 : 0.0;
-          for (int l = c; l < i; ++l) acc = fma(-s[kb + i][kb + l], mi[kb + l][kb + c], acc);
-          mi[kb + i][kb + c] = acc / s[kb + i][kb + i];
-        }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        s[kb + i][kb + 8 * h + c] = a[c];
+        mi[kb + i][kb + 8 * h + c] = r[c];
       }
     }
     __syncthreads();
@@ -168,9 +187,14 @@ __global__ void __launch_bounds__(256) potrf_diag_kernel(double* __restrict__ A,
         pv[q] = 0.0;
         if (e < rows * w) {
           const int i = r0 + e / w, c = e % w;
-          double acc = 0.0;
-          for (int l = 0; l <= c; ++l) acc = fma(s[i][kb + l], mi[kb + c][kb + l], acc);
-          pv[q] = acc;
+          double a0 = 0.0, a1 = 0.0;
+          int l = 0;
+          for (; l + 1 <= c; l += 2) {
+            a0 = fma(s[i][kb + l], mi[kb + c][kb + l], a0);
+            a1 = fma(s[i][kb + l + 1], mi[kb + c][kb + l + 1], a1);
+          }
+          if (l <= c) a0 = fma(s[i][kb + l], mi[kb + c][kb + l], a0);
+          pv[q] = a0 + a1;
         }
       }
       __syncthreads();
@@ -184,9 +208,16 @@ __global__ void __launch_bounds__(256) potrf_diag_kernel(double* __restrict__ A,
       for (int e = tid; e < rows * rows; e += blockDim.x) {
         const int i = r0 + e / rows, l = r0 + e % rows;
         if (l <= i) {
-          double acc = s[i][l];
-          for (int p = 0; p < w; ++p) acc = fma(-s[i][kb + p], s[l][kb + p], acc);
-          s[i][l] = acc;
+          double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+          int p = 0;
+          for (; p + 3 < w; p += 4) {
+            a0 = fma(s[i][kb + p], s[l][kb + p], a0);
+            a1 = fma(s[i][kb + p + 1], s[l][kb + p + 1], a1);
+            a2 = fma(s[i][kb + p + 2], s[l][kb + p + 2], a2);
+            a3 = fma(s[i][kb + p + 3], s[l][kb + p + 3], a3);
+          }
+          for (; p < w; ++p) a0 = fma(s[i][kb + p], s[l][kb + p], a0);
+          s[i][l] -= (a0 + a1) + (a2 + a3);
         }
       }
       __syncthreads();
@@ -200,9 +231,14 @@ __global__ void __launch_bounds__(256) potrf_diag_kernel(double* __restrict__ A,
     for (int e = tid; e < wi * i0; e += blockDim.x) {
       const int ii = e / i0, col = e % i0;
       const int k0 = (col / SB16) * SB16;
-      double acc = 0.0;
-      for (int k = k0; k < i0; ++k) acc = fma(s[i0 + ii][k], mi[k][col], acc);
-      mi[i0 + ii][col] = acc;
+      double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+      for (int k = k0; k < i0; k += 4) {        // i0 - k0 is a multiple of 16
+        a0 = fma(s[i0 + ii][k], mi[k][col], a0);
+        a1 = fma(s[i0 + ii][k + 1], mi[k + 1][col], a1);
+        a2 = fma(s[i0 + ii][k + 2], mi[k + 2][col], a2);
+        a3 = fma(s[i0 + ii][k + 3], mi[k + 3][col], a3);
+      }
+      mi[i0 + ii][col] = (a0 + a1) + (a2 + a3);
     }
     __syncthreads();
     double tv[3];
@@ -363,6 +399,33 @@ __global__ void colsumsq_final_kernel(const double* __restrict__ part, int npart
   h[j] = acc;
 }
 
+// Per host thread and device: a low-priority stream and events for the
+// inverse half of hinv_diag.
+struct SideStream {
+  int dev = -1;
+  bool ok = false;
+  cudaStream_t stream = nullptr;
+  std::vector<cudaEvent_t> ev;
+};
+static SideStream& side_stream(int events) {
+  thread_local SideStream ss[16];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  SideStream& x = ss[dev & 15];
+  if (x.dev != dev) {
+    int lo = 0, hi = 0;
+    cudaDeviceGetStreamPriorityRange(&lo, &hi);
+    x.ok = cudaStreamCreateWithPriority(&x.stream, cudaStreamNonBlocking, lo) == cudaSuccess;
+    x.dev = dev;
+  }
+  while (x.ok && (int)x.ev.size() < events) {
+    cudaEvent_t e;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) { x.ok = false; break; }
+    x.ev.push_back(e);
+  }
+  return x;
+}
+
 size_t hinv_workspace_doubles(int64_t n) {
   const int64_t parts = (n + kNormRows - 1) / kNormRows;
   return (size_t)(2 * n * n + parts * n + 64);
@@ -389,18 +452,27 @@ cudaError_t launch_hinv(const double* H, int64_t n, double alpha, double* h, dou
   damp_copy_kernel<<<dim3((unsigned)((n + 255) / 256), (unsigned)n), 256, 0, s>>>(H, n, damp, A);
   cudaMemsetAsync(M, 0, (size_t)n * n * sizeof(double), s);
   const int T = (int)((n + NB - 1) / NB);
+  // The inverse steps run on a lower-priority side stream: step I needs only
+  // panel I (column block I of L is final then; later trailing updates touch
+  // column blocks > K) and the diagonal inverse M_II, so they fill the SMs the
+  // one-CTA diagonal factorizations leave idle. Joined back before the norms.
+  SideStream& ss = side_stream(T + 1);
+  if (!ss.ok) return cudaErrorMemoryAllocation;
+  cudaEventRecord(ss.ev[T], s);
+  cudaStreamWaitEvent(ss.stream, ss.ev[T], 0);
   for (int K = 0; K < T; ++K) {
     potrf_diag_kernel<<<1, 256, tile_smem, s>>>(A, M, n, K, st);
     const int below = T - 1 - K;
-    if (below > 0) {
-      panel_kernel<<<below, 256, tile_smem, s>>>(A, M, n, K);
-      syrk_kernel<<<below * (below + 1) / 2, 256, tile_smem, s>>>(A, n, K);
-    }
+    if (below > 0) panel_kernel<<<below, 256, tile_smem, s>>>(A, M, n, K);
+    cudaEventRecord(ss.ev[K], s);
+    if (below > 0) syrk_kernel<<<below * (below + 1) / 2, 256, tile_smem, s>>>(A, n, K);
+    cudaStreamWaitEvent(ss.stream, ss.ev[K], 0);
+    if (K > 0) rowmult_kernel<<<K, 256, tile_smem, ss.stream>>>(M, n, K);
+    if (K < T - 1)
+      inv_update_kernel<<<dim3((unsigned)(T - 1 - K), (unsigned)(K + 1)), 256, tile_smem, ss.stream>>>(A, M, n, K);
   }
-  for (int I = 0; I < T; ++I) {
-    if (I > 0) rowmult_kernel<<<I, 256, tile_smem, s>>>(M, n, I);
-    if (I < T - 1) inv_update_kernel<<<dim3((unsigned)(T - 1 - I), (unsigned)(I + 1)), 256, tile_smem, s>>>(A, M, n, I);
-  }
+  cudaEventRecord(ss.ev[T], ss.stream);
+  cudaStreamWaitEvent(s, ss.ev[T], 0);
   colsumsq_partial_kernel<<<dim3((unsigned)((n + 255) / 256), (unsigned)parts), 256, 0, s>>>(M, n, part);
   colsumsq_final_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, (int)parts, n, h);
   count_launches(2 + T + 2 * (T - 1) + 2 * (T - 1) + 2);
