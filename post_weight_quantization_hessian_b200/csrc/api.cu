@@ -100,6 +100,21 @@ int finish(cudaStream_t s, const DevStatus* dst) {
   return SLIM_OK;
 }
 
+// Keep freed stream-ordered allocations in the device's default pool instead of
+// returning them to the driver at every synchronization, so repeated calls
+// that let the library allocate do not re-map gigabytes each time.
+void retain_pool_memory() {
+  thread_local int done_dev = -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev == done_dev) return;
+  cudaMemPool_t pool;
+  if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+    uint64_t keep = ~0ull;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+  }
+  done_dev = dev;
+}
+
 // Workspace holder: caller memory or a cudaMallocAsync'd block freed on scope exit.
 struct Workspace {
   uint8_t* p = nullptr;
@@ -112,6 +127,7 @@ struct Workspace {
       p = static_cast<uint8_t*>(ws);
       return SLIM_OK;
     }
+    retain_pool_memory();
     cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&p), need, st);
     if (e != cudaSuccess) { g_last_cuda_error = cudaGetErrorString(e); cudaGetLastError(); return SLIM_ENOMEM; }
     owned = true;

@@ -64,12 +64,19 @@ __global__ void damp_copy_kernel(const double* __restrict__ H, int64_t n, const 
 // ---------------------------------------------------------------- tile helpers
 // Load a (rows x cols) block at G (row-major, leading dim ld) into S[64][LDS],
 // either as is (S[r][c] = G[r][c]) or transposed (S[c][r] = G[r][c]); zero fill.
+// 256 threads, 16 elements each, all loads issued before the first store.
 __device__ __forceinline__ void load_tile(double (*S)[LDS], const double* G, int64_t ld, int rows, int cols,
                                           bool transpose) {
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
-    const double v = (r < rows && c < cols) ? G[(int64_t)r * ld + c] : 0.0;
-    if (transpose) S[c][r] = v; else S[r][c] = v;
+  double v[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int e = threadIdx.x + 256 * k, r = e / NB, c = e % NB;
+    v[k] = (r < rows && c < cols) ? G[(int64_t)r * ld + c] : 0.0;
+  }
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int e = threadIdx.x + 256 * k, r = e / NB, c = e % NB;
+    if (transpose) S[c][r] = v[k]; else S[r][c] = v[k];
   }
 }
 
@@ -121,10 +128,19 @@ __global__ void __launch_bounds__(256) potrf_diag_kernel(double* __restrict__ A,
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nb = blk_size(n, K);
   const int64_t off = (int64_t)K * NB * n + (int64_t)K * NB;
-  for (int e = tid; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
-    s[r][c] = (r < nb && c < nb && c <= r) ? A[off + (int64_t)r * n + c] : 0.0;
-    mi[r][c] = (r == c) ? 1.0 : 0.0;
+  {
+    double v[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int e = tid + 256 * k, r = e / NB, c = e % NB;
+      v[k] = (r < nb && c < nb && c <= r) ? A[off + (int64_t)r * n + c] : 0.0;
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int e = tid + 256 * k, r = e / NB, c = e % NB;
+      s[r][c] = v[k];
+      mi[r][c] = (r == c) ? 1.0 : 0.0;
+    }
   }
   __syncthreads();
   for (int kb = 0; kb < nb; kb += SB16) {

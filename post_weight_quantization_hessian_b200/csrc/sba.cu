@@ -322,25 +322,6 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           ++it;
           if (++st == S) { st = 0; ph ^= 1; }
         }
-        // warm L2 with what this tile needs next: the following phase-A slice, or the next delta step
-        auto prefetch = [&](const ItemGeom& g, int a, int b) {
-          for (int c = a; c < b; ++c) {
-            Chunk ch;
-            chunk_at(p, g, c, ch);
-            tma_prefetch_l2(&tm.x, ch.xcol, xrow);
-            if (ch.which == 0) {
-              tma_prefetch_l2(&tm.wb, ch.bcol, brow);
-              tma_prefetch_l2(&tm.e0, ch.bcol, brow);
-            } else {
-              tma_prefetch_l2(ch.which == 1 ? (const void*)&tm.dp : (const void*)&tm.dm, ch.bcol, brow);
-            }
-          }
-        };
-        if (step == 0) {
-          prefetch(geo, c1, min(p.nA, c1 + (c1 - c0)));
-        } else if (step + 1 < p.P) {
-          prefetch(item_geom(p, s_order, step + 1), 0, p.nD);
-        }
         return true;
       });
       // let every issued copy land before the CTA can exit

@@ -16,8 +16,15 @@
 // (lanes over elements): codes at the chosen tau, bytes to shared memory, then
 // the group's g*b/32 little-endian words.
 //
-// Cost: about 25 fp64 operations per (weight, tau) plus one IEEE division;
-// ALU-bound (the HBM traffic is ~4.3 bytes per weight).
+// The quotient w / s must be the correctly rounded one (the codes are
+// rint(w / s + z0)). Per candidate, the lane takes y = 1/s with the IEEE
+// division once, then per element Markstein's final division step (P.
+// Markstein, IBM J. Res. Dev. 34(1), 1990): q0 = w*y, r = fma(-q0, s, w),
+// q = fma(r, y, q0), which is the correctly rounded w/s when y = RN(1/s) and
+// nothing overflows or underflows (weights and scales come from fp32 values).
+//
+// Cost: about 12 fp64 operations per (weight, tau); ALU-bound (the HBM traffic
+// is ~4.3 bytes per weight).
 #include <cstdint>
 #include "common.cuh"
 
@@ -103,11 +110,14 @@ sqc_kernel(const float* __restrict__ W, int64_t m, int64_t n, const double* __re
       for (int t = lane; t < n_tau; t += 32) {
         const double tau = (n_tau == 1) ? 1.0 : (1.0 - lam) + ((2.0 * lam) * (double)t) / (double)(n_tau - 1);
         const double s = tau * s0;
+        const double y = 1.0 / s;
         double es = 0.0, eu = 0.0;
 #pragma unroll 4
         for (int j = 0; j < G; ++j) {
           const double wj = s_w[wib][j];
-          double q = rint(wj / s + z0);
+          const double q0 = wj * y;
+          const double quot = fma(fma(-q0, s, wj), y, q0);   // = RN(wj / s)
+          double q = rint(quot + z0);
           q = fmin(fmax(q, 0.0), qmax);
           const double e = wj - s * (q - z0);
           const double v = s_d[wib][j] * (e * e);

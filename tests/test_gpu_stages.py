@@ -119,3 +119,17 @@ def test_sba_search(kw):
         assert np.array_equal(bits.cpu().numpy(), ref.bits.astype(np.uint8))
     b = bits.cpu().numpy().astype(int)
     assert b.sum() == s.k * s.avg_bits
+
+
+def test_sqc_larger_layer():
+    """1M weights x 50 candidates: every quotient of the calibration loop exercised."""
+    s = spec(m=1024, n=1024, group=64, avg_bits=3, seed=21)
+    W = syn.make_weight(s)
+    h = np.random.default_rng(21).uniform(0.05, 1.0, s.n)
+    bits = balanced_bits(s.k, s.avg_bits, 5, seed=21)
+    codes, scale, zero, tau = slim.slim_sqc(torch.from_numpy(W).cuda(), torch.from_numpy(h).cuda(),
+                                            torch.from_numpy(bits).cuda(), s.group, s.avg_bits, 0.1, 50)
+    ref = O.sqc_calibrate(W, h, bits, s.group, 0.1, 50)
+    agree, tmis = compare_sqc(codes.cpu().numpy(), scale.cpu().numpy(), zero.cpu().numpy(), tau.cpu().numpy(),
+                              ref, bits, s.group, s.avg_bits)
+    assert agree >= 0.9999 and tmis == 0, (agree, tmis)
