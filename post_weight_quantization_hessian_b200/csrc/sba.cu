@@ -149,10 +149,10 @@ constexpr int SB_BM = 128;        // tokens per tile (TMEM lanes)
 constexpr int SB_BN = 128;        // outputs per tile (one TMEM slot: y and d, 128 columns each)
 constexpr int SB_BK = 64;         // K elements per box (128 bytes of fp16)
 constexpr int SB_BOX = SB_BM * SB_BK * 2;  // 16 KB
-constexpr int SB_STAGE = 3 * SB_BOX;       // X, B1, B2
-constexpr int SB_BAND = 32;                // token tiles per raster band
+constexpr int SB_STAGE = 4 * SB_BOX;       // X(token tile 0), X(token tile 1), B1, B2
+constexpr int SB_BAND = 16;                // token-tile pairs per raster band
 constexpr int SB_MAX_K = 1024;
-constexpr int SB_EPI_WARPS = 8;            // two per TMEM lane quadrant, 64 columns each
+constexpr int SB_EPI_WARPS = 8;            // warps 2..5 read slot 0, warps 6..9 slot 1
 constexpr int SB_THREADS = 64 + 32 * SB_EPI_WARPS;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kC1 = kLog2e * kOpUnscale;  // exponent scale for accumulator (x 2^8) units
@@ -164,10 +164,10 @@ struct SbaTmaps {
 struct SbaParams {
   int64_t N, m, n;
   int g, k, P, ksplit;
-  int n_tt, n_ot, stages;
-  int nA, nD;             // chunks of phase A and of one delta step
+  int n_tt, n_tp, n_ot, stages;  // token tiles, token-tile pairs, output tiles
+  int nA, nD;                    // chunks of phase A and of one delta step
   const int32_t* order;
-  float* part;            // [n_tt][n_ot][F][128], F = 2 + 2P
+  float* part;                   // [n_tt][n_ot][F][128], F = 2 + 2P
   DevStatus* st;
 };
 
@@ -176,48 +176,10 @@ struct Chunk {
   int which;  // 0: phase A (Wb, E0); 1: Dp; 2: Dm
 };
 
-// Work tile u -> (token tile, output tile), raster bands of SB_BAND token tiles.
-__device__ __forceinline__ void tile_decode(const SbaParams& p, int u, int& tt, int& ot) {
-  const int band_start = (u / (SB_BAND * p.n_ot)) * SB_BAND;
-  const int bc = (p.n_tt - band_start < SB_BAND) ? p.n_tt - band_start : SB_BAND;
-  const int r = u - band_start * p.n_ot;
-  ot = r / bc;
-  tt = band_start + (r - ot * bc);
-}
-
-// The MMA issue order of one CTA's T tiles, shared by the TMA producer and the
-// MMA issuer. Tile i alternates between the two TMEM slots. Phase A of tile i
-// is cut into slices placed before each delta step of tile i-1, so the tensor
-// pipe keeps busy while the epilogue digests tile i-1's candidates:
-//   A(T0) | A(T1) slice, D1(T0), A(T1) slice, D2(T0), ... | A(T2) slice, D1(T1), ... | ..., D_{P-1}(T_last)
-// f(tile, step, chunk_begin, chunk_end, item_chunks) is called once per slice
-// of an item (step 0: phase A, nA chunks; step p: delta p, nD chunks); it
-// returns false to abort the walk.
-template <class F>
-__device__ __forceinline__ bool walk_schedule(const SbaParams& p, int T, F&& f) {
-  const int steps = p.P - 1;
-  for (int i = 0; i <= T; ++i) {
-    const bool hasA = i < T, hasD = i > 0 && steps > 0;
-    if (!hasD) {
-      if (hasA && !f(i, 0, 0, p.nA, p.nA)) return false;
-      continue;
-    }
-    int a_done = 0;
-    for (int s = 1; s <= steps; ++s) {
-      if (hasA) {
-        const int a_to = (int)((int64_t)s * p.nA / steps);
-        if (a_to > a_done && !f(i, 0, a_done, a_to, p.nA)) return false;
-        a_done = a_to;
-      }
-      if (!f(i - 1, s, 0, p.nD, p.nD)) return false;
-    }
-  }
-  return true;
-}
-
-// Per-item chunk geometry without divisions in the chunk loop. Phase A chunk
-// c: K box c >> (ksplit - 1), X half c & (ksplit - 1). Delta chunk c: group
-// c / per_group (promoted first), then K box and X half within the group.
+// Per-item chunk geometry without divisions in the chunk loop. Step 0 is phase
+// A (y = X Wb^T, d = X E0^T over K = n; chunk c is K box c >> (ksplit - 1),
+// X half c & (ksplit - 1)); step p >= 1 adds the promoted group order[p-1]
+// (Dp) and the demoted group order[k-p] (Dm), promoted chunks first.
 struct ItemGeom {
   int step, ks_shift, per_group, col_up, col_dn, k16_lo_up, k16_lo_dn, k16_n;
 };
@@ -256,34 +218,48 @@ __device__ __forceinline__ void chunk_at(const SbaParams& p, const ItemGeom& g, 
   ch.xcol = ch.bcol + (sx ? (int)p.n : 0);
 }
 
+// Work unit u -> (token-tile pair, output tile); raster bands of SB_BAND pairs.
+__device__ __forceinline__ void unit_decode(const SbaParams& p, int u, int& tp, int& ot) {
+  const int band_start = (u / (SB_BAND * p.n_ot)) * SB_BAND;
+  const int bc = (p.n_tp - band_start < SB_BAND) ? p.n_tp - band_start : SB_BAND;
+  const int r = u - band_start * p.n_ot;
+  ot = r / bc;
+  tp = band_start + (r - ot * bc);
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
+// One work unit is two token tiles (TMEM slots 0 and 1) against one output tile:
+// every weight-side box feeds both slots' MMAs, so per output tile the kernel
+// moves about a third fewer bytes than with one token tile.
+//   warp 0      TMA producer (4 boxes per phase-A chunk, 3 per delta chunk)
+//   warp 1      TMEM owner (512 columns) and MMA issuer: phase A as N = 256 MMAs
+//               (Wb and E0 boxes adjacent; y and d adjacent in TMEM), delta steps
+//               as N = 128 MMAs into d, in place
+//   warps 2..9  epilogue, four per slot, one token row per thread, 128 columns
 __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_constant__ SbaTmaps tm, SbaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * SB_STAGE);
   uint64_t* empty = full + S;
-  uint64_t* afull = empty + S;   // [2] item accumulated in TMEM slot s
-  uint64_t* afree = afull + 2;   // [2] epilogue done with slot s's last item
+  uint64_t* afull = empty + S;   // [2] step accumulated in TMEM slot s
+  uint64_t* afree = afull + 2;   // [2] epilogue done reading slot s
   uint64_t* done = afree + 2;
-  uint64_t* xbar = done + 1;     // [4] column-half exchange, one per TMEM lane quadrant (64 threads)
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(xbar + 4);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-  float* xbuf = reinterpret_cast<float*>(tslot + 2);            // [2][4][2][3][32] half-to-half exchange
-  int32_t* s_order = reinterpret_cast<int32_t*>(xbuf + 2 * 4 * 2 * 3 * 32);
+  int32_t* s_order = reinterpret_cast<int32_t*>(tslot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int c = threadIdx.x; c < p.k; c += blockDim.x) s_order[c] = p.order[c];
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&afull[s], 1); mbar_init(&afree[s], SB_EPI_WARPS); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&afull[s], 1); mbar_init(&afree[s], SB_EPI_WARPS / 2); }
     mbar_init(done, 1);
-    for (int qq = 0; qq < 4; ++qq) mbar_init(&xbar[qq], 64);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -291,39 +267,42 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tslot;
-  const int tiles = p.n_tt * p.n_ot;
-  const int T = (tiles > (int)blockIdx.x) ? (tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  const int units = p.n_tp * p.n_ot;
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t it = 0;      // chunks issued (for the final drain)
-      int st = 0;           // stage ring position and its phase bit
+      uint32_t it = 0;
+      int st = 0;
       uint32_t ph = 0;
-      walk_schedule(p, T, [&](int ti, int step, int c0, int c1, int) -> bool {
-        int tt, ot;
-        tile_decode(p, (int)blockIdx.x + ti * (int)gridDim.x, tt, ot);
-        const ItemGeom geo = item_geom(p, s_order, step);
-        const int brow = ot * SB_BN, xrow = tt * SB_BM;
-        for (int c = c0; c < c1; ++c) {
-          Chunk ch;
-          chunk_at(p, geo, c, ch);
-          if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, p.st, 200 + st)) return false;
-          uint8_t* sb = smem + st * SB_STAGE;
-          mbar_arrive_expect_tx(&full[st], (ch.which == 0 ? 3 : 2) * SB_BOX);
-          tma_load_2d(sb, &tm.x, &full[st], ch.xcol, xrow);
-          if (ch.which == 0) {
-            tma_load_2d(sb + SB_BOX, &tm.wb, &full[st], ch.bcol, brow);
-            tma_load_2d(sb + 2 * SB_BOX, &tm.e0, &full[st], ch.bcol, brow);
-          } else {
-            tma_load_2d(sb + SB_BOX, ch.which == 1 ? (const void*)&tm.dp : (const void*)&tm.dm, &full[st], ch.bcol,
-                        brow);
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int tp, ot;
+        unit_decode(p, u, tp, ot);
+        const int xrow0 = 2 * tp * SB_BM, xrow1 = xrow0 + SB_BM, brow = ot * SB_BN;
+        for (int step = 0; step < p.P && ok; ++step) {
+          const ItemGeom geo = item_geom(p, s_order, step);
+          const int nch = step == 0 ? p.nA : p.nD;
+          for (int c = 0; c < nch; ++c) {
+            Chunk ch;
+            chunk_at(p, geo, c, ch);
+            if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, p.st, 200 + st)) { ok = false; break; }
+            uint8_t* sb = smem + st * SB_STAGE;
+            mbar_arrive_expect_tx(&full[st], (ch.which == 0 ? 4 : 3) * SB_BOX);
+            tma_load_2d(sb, &tm.x, &full[st], ch.xcol, xrow0);
+            tma_load_2d(sb + SB_BOX, &tm.x, &full[st], ch.xcol, xrow1);
+            if (ch.which == 0) {
+              tma_load_2d(sb + 2 * SB_BOX, &tm.wb, &full[st], ch.bcol, brow);
+              tma_load_2d(sb + 3 * SB_BOX, &tm.e0, &full[st], ch.bcol, brow);
+            } else {
+              tma_load_2d(sb + 2 * SB_BOX, ch.which == 1 ? (const void*)&tm.dp : (const void*)&tm.dm, &full[st],
+                          ch.bcol, brow);
+            }
+            ++it;
+            if (++st == S) { st = 0; ph ^= 1; }
           }
-          ++it;
-          if (++st == S) { st = 0; ph ^= 1; }
         }
-        return true;
-      });
+      }
       // let every issued copy land before the CTA can exit
       for (uint32_t j = (it > (uint32_t)S ? it - S : 0); j < it; ++j) {
         uint64_t t0 = global_ns();
@@ -336,83 +315,78 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
       constexpr uint32_t idesc = idesc_f16_f32(SB_BM, SB_BN, false, false);
       constexpr uint32_t idesc2 = idesc_f16_f32(SB_BM, 2 * SB_BN, false, false);
       int st = 0;
-      uint32_t ph = 0;
-      uint32_t cnt[2] = {0, 0};
-      walk_schedule(p, T, [&](int ti, int step, int c0, int c1, int nitem) -> bool {
-        const int slot = ti & 1;
-        if (c0 == 0) {
-          if (!mbar_wait(&afree[slot], (cnt[slot] & 1) ^ 1, abort_flag, p.st, 220 + slot)) return false;
+      uint32_t ph = 0, cnt = 0;
+      bool ok = true;
+      const uint32_t ty0 = tbase, ty1 = tbase + 256;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        for (int step = 0; step < p.P && ok; ++step) {
+          if (!mbar_wait(&afree[0], (cnt & 1) ^ 1, abort_flag, p.st, 220) ||
+              !mbar_wait(&afree[1], (cnt & 1) ^ 1, abort_flag, p.st, 221)) { ok = false; break; }
           tc_fence_after();
-        }
-        const ItemGeom geo = item_geom(p, s_order, step);
-        const uint32_t ty = tbase + slot * 256, td = ty + 128;
-        for (int c = c0; c < c1; ++c) {
-          Chunk ch;
-          chunk_at(p, geo, c, ch);
-          if (!mbar_wait(&full[st], ph, abort_flag, p.st, 230 + st)) return false;
-          tc_fence_after();
-          const uint32_t xa = smem_u32(smem + st * SB_STAGE);
-          const uint64_t ad0 = sdesc_sw128(xa, 16, 1024);
-          const uint64_t b10 = sdesc_sw128(xa + SB_BOX, 16, 1024);
-          if (ch.which == 0) {
-            // the Wb and E0 boxes are adjacent (256 B-operand rows), and so are y and d in TMEM:
-            // one N = 256 MMA per k16 step writes both accumulators
+          const ItemGeom geo = item_geom(p, s_order, step);
+          const int nch = step == 0 ? p.nA : p.nD;
+          for (int c = 0; c < nch; ++c) {
+            Chunk ch;
+            chunk_at(p, geo, c, ch);
+            if (!mbar_wait(&full[st], ph, abort_flag, p.st, 230 + st)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t xa = smem_u32(smem + st * SB_STAGE);
+            const uint64_t a0 = sdesc_sw128(xa, 16, 1024);
+            const uint64_t a1 = sdesc_sw128(xa + SB_BOX, 16, 1024);
+            const uint64_t b0 = sdesc_sw128(xa + 2 * SB_BOX, 16, 1024);
+            // advancing 32 bytes along K = +2 in the descriptor's 16-byte start-address field
+            if (ch.which == 0) {
 #pragma unroll
-            for (int k16 = 0; k16 < 4; ++k16) {
-              const uint32_t acc = (c > 0 || k16 > 0) ? 1u : 0u;
-              // advancing 32 bytes along K = +2 in the descriptor's 16-byte start-address field
-              tc_mma_f16(ty, ad0 + 2 * k16, b10 + 2 * k16, idesc2, acc);
+              for (int k16 = 0; k16 < 4; ++k16) {
+                const uint32_t acc = (c > 0 || k16 > 0) ? 1u : 0u;
+                tc_mma_f16(ty0, a0 + 2 * k16, b0 + 2 * k16, idesc2, acc);
+                tc_mma_f16(ty1, a1 + 2 * k16, b0 + 2 * k16, idesc2, acc);
+              }
+            } else {
+              for (int k16 = ch.k16_lo; k16 < ch.k16_hi; ++k16) {
+                tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, 1u);
+                tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, 1u);
+              }
             }
-          } else {
-            for (int k16 = ch.k16_lo; k16 < ch.k16_hi; ++k16)
-              tc_mma_f16(td, ad0 + 2 * k16, b10 + 2 * k16, idesc, 1u);
+            tc_commit(&empty[st]);
+            if (++st == S) { st = 0; ph ^= 1; }
           }
-          tc_commit(&empty[st]);
-          if (++st == S) { st = 0; ph ^= 1; }
+          if (!ok) break;
+          tc_commit(&afull[0]);
+          tc_commit(&afull[1]);
+          ++cnt;
         }
-        if (c1 == nitem) {
-          tc_commit(&afull[slot]);
-          ++cnt[slot];
-        }
-        return true;
-      });
+      }
       tc_commit(done);
       uint64_t t0 = global_ns();
       while (!mbar_try_wait(done, 0) && global_ns() - t0 < kWaitLimitNs) {}
     }
   } else {
-    // ------------------------------------------------ epilogue: 8 warps, token row per lane, 64 columns per warp
+    // ------------------------------------------------ epilogue: slot (warp-2)/4, token row per lane
+    const int slot = (warp - 2) >> 2;
     const int q = warp & 3;                 // TMEM lane quadrant this warp may access
-    const int hf = (warp - 2) >> 2;         // which 64 of the tile's 128 columns
     const int r = q * 32 + lane;            // token row inside the tile
     const int F = 2 + 2 * p.P;
-    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    uint32_t cnt[2] = {0, 0};
-    int xc = 0;                             // exchange counter (double-buffered xbuf)
-    auto xb = [&](int buf, int half, int val) -> float& { return xbuf[((((buf * 4) + q) * 2 + half) * 3 + val) * 32 + lane]; };
-    // both 32-lane halves of quadrant q arrive, then wait (bounded) for exchange xc's phase
-    auto xsync = [&]() -> bool {
-      mbar_arrive(&xbar[q]);
-      return mbar_wait(&xbar[q], xc & 1, abort_flag, p.st, 250 + q);
-    };
+    const uint32_t ty = tbase + ((uint32_t)(q * 32) << 16) + slot * 256, td = ty + 128;
+    uint32_t cnt = 0;
     bool ok = true;
-    for (int ti = 0; ti < T && ok; ++ti) {
-      const int slot = ti & 1;
-      int tt, ot;
-      tile_decode(p, (int)blockIdx.x + ti * (int)gridDim.x, tt, ot);
-      const int64_t col0 = (int64_t)ot * SB_BN + hf * 64;
-      const int nvalid = (int)((p.m - col0) < 0 ? 0 : ((p.m - col0) > 64 ? 64 : (p.m - col0)));
-      float* outp = p.part + ((size_t)tt * p.n_ot + ot) * F * SB_BM + r;
-      const uint32_t ty = tbase + lane_off + slot * 256 + hf * 64, td = ty + 128;
-      float Mt = 0.f, syt = 0.f;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      int tp, ot;
+      unit_decode(p, u, tp, ot);
+      const int tt = 2 * tp + slot;
+      const bool have = tt < p.n_tt;        // the second tile of an odd pair is padding
+      const int64_t col0 = (int64_t)ot * SB_BN;
+      const int nvalid = (int)((p.m - col0) > SB_BN ? SB_BN : (p.m - col0));
+      float* outp = p.part + ((size_t)(have ? tt : 0) * p.n_ot + ot) * F * SB_BM + r;
+      float Mt = 0.f;
       for (int step = 0; step < p.P; ++step) {
-        if (!mbar_wait(&afull[slot], cnt[slot] & 1, abort_flag, p.st, 240 + slot)) { ok = false; break; }
+        if (!mbar_wait(&afull[slot], cnt & 1, abort_flag, p.st, 240 + slot)) { ok = false; break; }
         tc_fence_after();
         float sq0 = 0.f, sq1 = 0.f, a0 = 0.f, a1 = 0.f, sy0 = 0.f, sy1 = 0.f;
         if (step == 0) {
           float mx = -3.0e38f;
 #pragma unroll 1
-          for (int cc = 0; cc < 2; ++cc) {
+          for (int cc = 0; cc < 4; ++cc) {
             uint32_t yv[32];
             tmem_ld32(ty + cc * 32, yv);
             tc_wait_ld();
@@ -420,14 +394,9 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
             for (int v = 0; v < 32; ++v)
               if (cc * 32 + v < nvalid) mx = fmaxf(mx, __uint_as_float(yv[v]));
           }
-          // tile maximum: combine with the partner warp holding the other 64 columns
-          xb(xc & 1, hf, 0) = mx;
-          if (!xsync()) { ok = false; break; }
-          mx = fmaxf(mx, xb(xc & 1, hf ^ 1, 0));
-          ++xc;
           const float mb = -mx * kC1;
 #pragma unroll 1
-          for (int cc = 0; cc < 2; ++cc) {
+          for (int cc = 0; cc < 4; ++cc) {
             uint32_t yv[32], dv[32];
             tmem_ld32(ty + cc * 32, yv);
             tmem_ld32(td + cc * 32, dv);
@@ -453,7 +422,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           Mt = mx;
         } else {
 #pragma unroll 1
-          for (int cc = 0; cc < 2; ++cc) {
+          for (int cc = 0; cc < 4; ++cc) {
             uint32_t ev[32], dv[32];
             tmem_ld32(ty + cc * 32, ev);
             tmem_ld32(td + cc * 32, dv);
@@ -472,28 +441,15 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&afree[slot]);
-        ++cnt[slot];
-        // combine the two column halves; half 0 writes this tile's partial statistics
-        float sy = sy0 + sy1, sq = sq0 + sq1, a = a0 + a1;
-        if (hf == 1) {
-          xb(xc & 1, 1, 0) = sy;
-          xb(xc & 1, 1, 1) = sq;
-          xb(xc & 1, 1, 2) = a;
-        }
-        if (!xsync()) { ok = false; break; }
-        if (hf == 0) {
-          sy += xb(xc & 1, 1, 0);
-          sq += xb(xc & 1, 1, 1);
-          a += xb(xc & 1, 1, 2);
+        ++cnt;
+        if (have) {
           if (step == 0) {
-            syt = sy;
             outp[0] = Mt * kOpUnscale;
-            outp[SB_BM] = syt;
+            outp[SB_BM] = sy0 + sy1;
           }
-          outp[(size_t)(2 + 2 * step) * SB_BM] = sq;
-          outp[(size_t)(3 + 2 * step) * SB_BM] = a * kOpUnscale;
+          outp[(size_t)(2 + 2 * step) * SB_BM] = sq0 + sq1;
+          outp[(size_t)(3 + 2 * step) * SB_BM] = (a0 + a1) * kOpUnscale;
         }
-        ++xc;
       }
     }
   }
@@ -568,7 +524,7 @@ __global__ void sba_final_kernel(const double* __restrict__ kl_part, int n_tt, i
 
 // ---------------------------------------------------------------- host side
 struct SbaPlan {
-  int k, P, ksplit, n_tt, n_ot, stages, nA, nD;
+  int k, P, ksplit, n_tt, n_tp, n_ot, stages, nA, nD;
   size_t off_wb, off_e0, off_dp, off_dm, off_xc, off_part, off_klp, total;
   size_t smem;
 };
@@ -582,6 +538,7 @@ SbaPlan sba_plan(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
   pl.ksplit = xdtype == 1 ? 1 : 2;
   pl.n_tt = (int)((N + SB_BM - 1) / SB_BM);
   pl.n_ot = (int)((m + SB_BN - 1) / SB_BN);
+  pl.n_tp = (pl.n_tt + 1) / 2;
   pl.nA = (int)((n + SB_BK - 1) / SB_BK) * pl.ksplit;
   pl.nD = 2 * (group >= 64 ? group / 64 : 1) * pl.ksplit;
   const size_t wbytes = (size_t)m * n * 2;
@@ -594,8 +551,8 @@ SbaPlan sba_plan(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
   pl.off_part = off; off = align256(off + (size_t)pl.n_tt * pl.n_ot * (2 + 2 * pl.P) * SB_BM * sizeof(float));
   pl.off_klp = off; off = align256(off + (size_t)pl.P * pl.n_tt * sizeof(double));
   pl.total = off;
-  const size_t fixed = 1024 + 512 + 2 * 4 * 2 * 3 * 32 * sizeof(float) + (size_t)pl.k * 4 + 64;
-  int st = 4;
+  const size_t fixed = 1024 + 512 + (size_t)pl.k * 4 + 64;
+  int st = 3;
   while (st > 2 && fixed + (size_t)st * SB_STAGE > 227 * 1024) --st;
   pl.stages = st;
   pl.smem = fixed + (size_t)st * SB_STAGE;
@@ -647,12 +604,12 @@ cudaError_t launch_sba(const float* W, int64_t m, int64_t n, const void* X, int 
 
   SbaParams p;
   p.N = N; p.m = m; p.n = n; p.g = group; p.k = pl.k; p.P = pl.P; p.ksplit = pl.ksplit;
-  p.n_tt = pl.n_tt; p.n_ot = pl.n_ot; p.stages = pl.stages; p.nA = pl.nA; p.nD = pl.nD;
+  p.n_tt = pl.n_tt; p.n_tp = pl.n_tp; p.n_ot = pl.n_ot; p.stages = pl.stages; p.nA = pl.nA; p.nD = pl.nD;
   p.order = order; p.part = part; p.st = st;
   cudaError_t e = cudaFuncSetAttribute(sba_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
   if (e != cudaSuccess) return e;
-  const int tiles = pl.n_tt * pl.n_ot;
-  const int grid = tiles < num_sms ? tiles : num_sms;
+  const int units = pl.n_tp * pl.n_ot;
+  const int grid = units < num_sms ? units : num_sms;
   if (kev) cudaEventRecord(kev[0], s);
   sba_score_kernel<<<grid, SB_THREADS, pl.smem, s>>>(tm, p);
   if (kev) cudaEventRecord(kev[1], s);
