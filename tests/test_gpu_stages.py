@@ -43,7 +43,7 @@ def test_hessian_f32():
 
 
 # ---------------------------------------------------------------- hinv_diag
-@pytest.mark.parametrize("n", [320, 96, 1056])
+@pytest.mark.parametrize("n", [320, 96, 1056, 200, 1000])   # 200, 1000: padded to a multiple of 32 internally
 def test_hinv_diag(n):
     rng = np.random.default_rng(n)
     X = rng.standard_normal((4 * n, n))
