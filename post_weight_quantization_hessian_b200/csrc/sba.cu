@@ -152,7 +152,7 @@ constexpr int SB_BOX = SB_BM * SB_BK * 2;  // 16 KB
 constexpr int SB_STAGE = 4 * SB_BOX;       // X(token tile 0), X(token tile 1), B1, B2
 constexpr int SB_BAND = 16;                // token-tile pairs per raster band
 constexpr int SB_MAX_K = 1024;
-constexpr int SB_EPI_WARPS = 8;            // warps 2..5 read slot 0, warps 6..9 slot 1
+constexpr int SB_EPI_WARPS = 16;           // warps 2..9 read slot 0, warps 10..17 slot 1 (two per row)
 constexpr int SB_THREADS = 64 + 32 * SB_EPI_WARPS;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kC1 = kLog2e * kOpUnscale;  // exponent scale for accumulator (x 2^8) units
@@ -240,7 +240,11 @@ __device__ __forceinline__ float ex2(float x) {
 //   warp 1      TMEM owner (512 columns) and MMA issuer: phase A as N = 256 MMAs
 //               (Wb and E0 boxes adjacent; y and d adjacent in TMEM), delta steps
 //               as N = 128 MMAs into d, in place
-//   warps 2..9  epilogue, four per slot, one token row per thread, 128 columns
+//   warps 2..17 epilogue, eight per slot: two threads per token row, 64 columns
+//               each. A thread copies its d columns to registers and releases
+//               the accumulator before computing, so the next candidate's MMA
+//               overlaps the epilogue's exponentials; the two halves of a row
+//               combine their row maximum and sums through shared memory.
 __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_constant__ SbaTmaps tm, SbaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -250,9 +254,11 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
   uint64_t* afull = empty + S;   // [2] step accumulated in TMEM slot s
   uint64_t* afree = afull + 2;   // [2] epilogue done reading slot s
   uint64_t* done = afree + 2;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* xbar = done + 1;     // [8 row groups (slot, quadrant)][4]: max of half 0, max of half 1, sums x2
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(xbar + 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   int32_t* s_order = reinterpret_cast<int32_t*>(tslot + 2);
+  float* s_x = reinterpret_cast<float*>(s_order + ((p.k + 3) & ~3));  // [2 slots][128 rows][8]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int c = threadIdx.x; c < p.k; c += blockDim.x) s_order[c] = p.order[c];
@@ -260,6 +266,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int s = 0; s < 2; ++s) { mbar_init(&afull[s], 1); mbar_init(&afree[s], SB_EPI_WARPS / 2); }
     mbar_init(done, 1);
+    for (int b = 0; b < 32; ++b) mbar_init(&xbar[b], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -362,94 +369,111 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
       while (!mbar_try_wait(done, 0) && global_ns() - t0 < kWaitLimitNs) {}
     }
   } else {
-    // ------------------------------------------------ epilogue: slot (warp-2)/4, token row per lane
-    const int slot = (warp - 2) >> 2;
-    const int q = warp & 3;                 // TMEM lane quadrant this warp may access
-    const int r = q * 32 + lane;            // token row inside the tile
+    // ------------------------------------------------ epilogue
+    // warp e = warp - 2: slot e >> 3, column half h = (e >> 2) & 1, TMEM lane
+    // quadrant q = warp & 3 (the quadrant a warp may access); row r = 32 q + lane.
+    const int e = warp - 2;
+    const int slot = e >> 3, h = (e >> 2) & 1, q = warp & 3;
+    const int r = q * 32 + lane;
     const int F = 2 + 2 * p.P;
-    const uint32_t ty = tbase + ((uint32_t)(q * 32) << 16) + slot * 256, td = ty + 128;
-    uint32_t cnt = 0;
+    const uint32_t ty = tbase + ((uint32_t)(q * 32) << 16) + slot * 256 + h * 64, td = ty + 128;
+    float* xs = s_x + (slot * 128 + r) * 8;   // [0..3] even steps, [4..7] odd steps
+    uint64_t* xb = xbar + (slot * 4 + q) * 4;  // max h0, max h1, sums (even), sums (odd)
+    uint32_t cnt = 0, nunit = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++nunit) {
       int tp, ot;
       unit_decode(p, u, tp, ot);
       const int tt = 2 * tp + slot;
       const bool have = tt < p.n_tt;        // the second tile of an odd pair is padding
-      const int64_t col0 = (int64_t)ot * SB_BN;
-      const int nvalid = (int)((p.m - col0) > SB_BN ? SB_BN : (p.m - col0));
+      const int64_t col0 = (int64_t)ot * SB_BN + h * 64;
+      const int nvalid = (int)((p.m - col0) > 64 ? 64 : ((p.m - col0) > 0 ? (p.m - col0) : 0));
       float* outp = p.part + ((size_t)(have ? tt : 0) * p.n_ot + ot) * F * SB_BM + r;
       float Mt = 0.f;
       for (int step = 0; step < p.P; ++step) {
         if (!mbar_wait(&afull[slot], cnt & 1, abort_flag, p.st, 240 + slot)) { ok = false; break; }
         tc_fence_after();
-        float sq0 = 0.f, sq1 = 0.f, a0 = 0.f, a1 = 0.f, sy0 = 0.f, sy1 = 0.f;
+        uint32_t v[64];
+        float sy = 0.f;
         if (step == 0) {
+          // y -> row maximum (both halves) -> e^(y - M) stored back in place of y
+          tmem_ld32(ty, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+          tmem_ld32(ty + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          tc_wait_ld();
           float mx = -3.0e38f;
-#pragma unroll 1
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t yv[32];
-            tmem_ld32(ty + cc * 32, yv);
-            tc_wait_ld();
 #pragma unroll
-            for (int v = 0; v < 32; ++v)
-              if (cc * 32 + v < nvalid) mx = fmaxf(mx, __uint_as_float(yv[v]));
-          }
+          for (int j = 0; j < 64; ++j)
+            if (j < nvalid) mx = fmaxf(mx, __uint_as_float(v[j]));
+          xs[h ? 0 : 4] = mx;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&xb[h]);
+          if (!mbar_wait(&xb[h ^ 1], nunit & 1, abort_flag, p.st, 250 + slot)) { ok = false; break; }
+          mx = fmaxf(mx, xs[h ? 4 : 0]);
           const float mb = -mx * kC1;
-#pragma unroll 1
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t yv[32], dv[32];
-            tmem_ld32(ty + cc * 32, yv);
-            tmem_ld32(td + cc * 32, dv);
-            tc_wait_ld();
 #pragma unroll
-            for (int v = 0; v < 32; v += 2) {
-              const bool ok0 = cc * 32 + v < nvalid, ok1 = cc * 32 + v + 1 < nvalid;
-              const float ey0 = ok0 ? ex2(fmaf(__uint_as_float(yv[v]), kC1, mb)) : 0.f;
-              const float ey1 = ok1 ? ex2(fmaf(__uint_as_float(yv[v + 1]), kC1, mb)) : 0.f;
-              const float d0 = __uint_as_float(dv[v]), d1 = __uint_as_float(dv[v + 1]);
-              sy0 += ey0;
-              sy1 += ey1;
-              sq0 = fmaf(ey0, ex2(d0 * kC1), sq0);
-              sq1 = fmaf(ey1, ex2(d1 * kC1), sq1);
-              a0 = fmaf(ey0, d0, a0);
-              a1 = fmaf(ey1, d1, a1);
-              yv[v] = __float_as_uint(ey0);
-              yv[v + 1] = __float_as_uint(ey1);
-            }
-            tmem_st32(ty + cc * 32, yv);
+          for (int j = 0; j < 64; ++j) {
+            const float ey = (j < nvalid) ? ex2(fmaf(__uint_as_float(v[j]), kC1, mb)) : 0.f;
+            sy += ey;
+            v[j] = __float_as_uint(ey);
           }
+          tmem_st32(ty, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+          tmem_st32(ty + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
           tc_wait_st();
           Mt = mx;
-        } else {
-#pragma unroll 1
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t ev[32], dv[32];
-            tmem_ld32(ty + cc * 32, ev);
-            tmem_ld32(td + cc * 32, dv);
-            tc_wait_ld();
+        }
+        // this step's d to registers, then release the accumulator (except at the
+        // unit's last step: the next unit's first MMA overwrites e^(y - M))
+        tmem_ld32(td, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(td + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tc_wait_ld();
+        const bool last = step == p.P - 1;
+        if (!last) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afree[slot]);
+        }
+        float sq0 = 0.f, sq1 = 0.f, a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int v = 0; v < 32; v += 2) {
-              const float ey0 = __uint_as_float(ev[v]), ey1 = __uint_as_float(ev[v + 1]);
-              const float d0 = __uint_as_float(dv[v]), d1 = __uint_as_float(dv[v + 1]);
-              sq0 = fmaf(ey0, ex2(d0 * kC1), sq0);
-              sq1 = fmaf(ey1, ex2(d1 * kC1), sq1);
-              a0 = fmaf(ey0, d0, a0);
-              a1 = fmaf(ey1, d1, a1);
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t ev[8];
+          tmem_ld8(ty + cc * 8, ev);
+          tc_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; j += 2) {
+            const float ey0 = __uint_as_float(ev[j]), ey1 = __uint_as_float(ev[j + 1]);
+            const float d0 = __uint_as_float(v[cc * 8 + j]), d1 = __uint_as_float(v[cc * 8 + j + 1]);
+            sq0 = fmaf(ey0, ex2(d0 * kC1), sq0);
+            sq1 = fmaf(ey1, ex2(d1 * kC1), sq1);
+            a0 = fmaf(ey0, d0, a0);
+            a1 = fmaf(ey1, d1, a1);
+          }
+        }
+        if (last) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afree[slot]);
+        }
+        // half 1 hands its sums to half 0, which writes the row's partials
+        const int par = cnt & 1;
+        float* xo = xs + 4 * par;
+        if (h == 1) {
+          xo[1] = sy;
+          xo[2] = sq0 + sq1;
+          xo[3] = a0 + a1;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&xb[2 + par]);
+        } else {
+          if (!mbar_wait(&xb[2 + par], (cnt >> 1) & 1, abort_flag, p.st, 252 + slot)) { ok = false; break; }
+          if (have) {
+            if (step == 0) {
+              outp[0] = Mt * kOpUnscale;
+              outp[SB_BM] = sy + xo[1];
             }
+            outp[(size_t)(2 + 2 * step) * SB_BM] = (sq0 + sq1) + xo[2];
+            outp[(size_t)(3 + 2 * step) * SB_BM] = ((a0 + a1) + xo[3]) * kOpUnscale;
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&afree[slot]);
         ++cnt;
-        if (have) {
-          if (step == 0) {
-            outp[0] = Mt * kOpUnscale;
-            outp[SB_BM] = sy0 + sy1;
-          }
-          outp[(size_t)(2 + 2 * step) * SB_BM] = sq0 + sq1;
-          outp[(size_t)(3 + 2 * step) * SB_BM] = (a0 + a1) * kOpUnscale;
-        }
       }
     }
   }
@@ -551,7 +575,7 @@ SbaPlan sba_plan(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
   pl.off_part = off; off = align256(off + (size_t)pl.n_tt * pl.n_ot * (2 + 2 * pl.P) * SB_BM * sizeof(float));
   pl.off_klp = off; off = align256(off + (size_t)pl.P * pl.n_tt * sizeof(double));
   pl.total = off;
-  const size_t fixed = 1024 + 512 + (size_t)pl.k * 4 + 64;
+  const size_t fixed = 1024 + 512 + 256 + (size_t)(pl.k + 4) * 4 + 64 + 2 * 128 * 8 * sizeof(float);
   int st = 3;
   while (st > 2 && fixed + (size_t)st * SB_STAGE > 227 * 1024) --st;
   pl.stages = st;
