@@ -318,45 +318,57 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
+    // The issuing thread shares its SM sub-partition with four busy epilogue
+    // warps, so its instruction stream per MMA is kept short: stage descriptors
+    // come from one base by adding whole stages in 16-byte units, and the
+    // 64-wide boxes' four K steps are unrolled.
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(SB_BM, SB_BN, false, false);
       constexpr uint32_t idesc2 = idesc_f16_f32(SB_BM, 2 * SB_BN, false, false);
+      constexpr uint64_t kStage16 = SB_STAGE / 16, kBox16 = SB_BOX / 16;
+      const uint64_t d_first = sdesc_sw128(smem_u32(smem), 16, 1024);  // start-address field never carries (< 256 KB)
+      uint64_t dcur = d_first;
       int st = 0;
       uint32_t ph = 0, cnt = 0;
       bool ok = true;
       const uint32_t ty0 = tbase, ty1 = tbase + 256;
+      const bool dfull = p.g >= 64;  // delta chunks are whole 64-wide boxes
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         for (int step = 0; step < p.P && ok; ++step) {
           if (!mbar_wait(&afree[0], (cnt & 1) ^ 1, abort_flag, p.st, 220) ||
               !mbar_wait(&afree[1], (cnt & 1) ^ 1, abort_flag, p.st, 221)) { ok = false; break; }
           tc_fence_after();
-          const ItemGeom geo = item_geom(p, s_order, step);
+          ItemGeom geo;
+          if (step > 0 && !dfull) geo = item_geom(p, s_order, step);
           const int nch = step == 0 ? p.nA : p.nD;
           for (int c = 0; c < nch; ++c) {
-            Chunk ch;
-            chunk_at(p, geo, c, ch);
             if (!mbar_wait(&full[st], ph, abort_flag, p.st, 230 + st)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t xa = smem_u32(smem + st * SB_STAGE);
-            const uint64_t a0 = sdesc_sw128(xa, 16, 1024);
-            const uint64_t a1 = sdesc_sw128(xa + SB_BOX, 16, 1024);
-            const uint64_t b0 = sdesc_sw128(xa + 2 * SB_BOX, 16, 1024);
+            const uint64_t a0 = dcur, a1 = dcur + kBox16, b0 = dcur + 2 * kBox16;
             // advancing 32 bytes along K = +2 in the descriptor's 16-byte start-address field
-            if (ch.which == 0) {
+            if (step == 0) {
 #pragma unroll
               for (int k16 = 0; k16 < 4; ++k16) {
                 const uint32_t acc = (c > 0 || k16 > 0) ? 1u : 0u;
                 tc_mma_f16(ty0, a0 + 2 * k16, b0 + 2 * k16, idesc2, acc);
                 tc_mma_f16(ty1, a1 + 2 * k16, b0 + 2 * k16, idesc2, acc);
               }
+            } else if (dfull) {
+#pragma unroll
+              for (int k16 = 0; k16 < 4; ++k16) {
+                tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, 1u);
+                tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, 1u);
+              }
             } else {
+              Chunk ch;
+              chunk_at(p, geo, c, ch);
               for (int k16 = ch.k16_lo; k16 < ch.k16_hi; ++k16) {
                 tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, 1u);
                 tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, 1u);
               }
             }
             tc_commit(&empty[st]);
-            if (++st == S) { st = 0; ph ^= 1; }
+            if (++st == S) { st = 0; ph ^= 1; dcur = d_first; } else { dcur += kStage16; }
           }
           if (!ok) break;
           tc_commit(&afull[0]);
