@@ -118,7 +118,8 @@ sqc_kernel(const float* __restrict__ W, int64_t m, int64_t n, const double* __re
           const double q0 = wj * y;
           const double quot = fma(fma(-q0, s, wj), y, q0);   // = RN(wj / s)
           double q = rint(quot + z0);
-          q = fmin(fmax(q, 0.0), qmax);
+          q = (q < 0.0) ? 0.0 : q;   // clamp by selects: the fp64 min/max are slower here
+          q = (q > qmax) ? qmax : q;
           const double e = wj - s * (q - z0);
           const double v = s_d[wib][j] * (e * e);
           if (s_msk[wib][j]) es += v; else eu += v;
