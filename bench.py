@@ -167,13 +167,26 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """Largest value over the ranks (the job's step time is its slowest rank's)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_spec(spec: syn.LayerSpec, rank: int, world: int) -> syn.LayerSpec:
+    """With N ranks every rank quantizes its own independent layer of the same shape
+    (replicas; no data-path collective), seeded by its rank."""
+    return spec if world == 1 else spec.replace(seed=spec.seed + 7919 * rank)
+
+
+def job_value(world: int, spec: syn.LayerSpec, ms_per_step: float) -> float:
+    """Whole-job throughput: the weights all ranks quantized per second (Mparam/s)."""
+    return world * spec.m * spec.n / (ms_per_step * 1e-3) / 1e6
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -238,8 +251,7 @@ def run_ours(args, spec, world, rank, local):
         build.build()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    if world > 1:
-        spec = spec.replace(seed=spec.seed + 7919 * rank)       # an independent layer per rank
+    spec = replica_spec(spec, rank, world)
     W = syn.make_weight(spec)
     Xh_pinned = torch.empty((spec.N, spec.n), dtype=torch.int16, pin_memory=True)
     syn.make_activations(spec, out=Xh_pinned.numpy().view(np.uint16))
@@ -277,7 +289,7 @@ def run_ours(args, spec, world, rank, local):
     launches = (slim.slim_launch_count() - n0) / args.steps
     step_ms = [a.elapsed_time(b) for a, b in ev]
     ms = max_over_ranks(statistics.mean(step_ms), world)
-    value = world * spec.m * spec.n / (ms * 1e-3) / 1e6
+    value = job_value(world, spec, ms)
     p_star = d["p_star"]
 
     # ---- end to end through the host-buffer entry point (pinned host memory)
@@ -302,7 +314,7 @@ def run_ours(args, spec, world, rank, local):
             e2e_ms.append(a.elapsed_time(b))
         barrier(world)
         ems = max_over_ranks(statistics.mean(e2e_ms), world)
-        e2e = {"value": world * spec.m * spec.n / (ems * 1e-3) / 1e6, "unit": UNIT,
+        e2e = {"value": job_value(world, spec, ems), "unit": UNIT,
                "h2d_bytes_per_step": int(Wn.nbytes + Xn.nbytes),
                "d2h_bytes_per_step": int(sum(o.nbytes for o in outs)), "ms_per_step": ems}
 
