@@ -233,6 +233,28 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): the epilogue handles two output
+// columns per instruction, which leaves more issue slots to the MMA thread on
+// the same SM sub-partition.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // One work unit is two token tiles (TMEM slots 0 and 1) against one output tile:
 // every weight-side box feeds both slots' MMAs, so per output tile the kernel
 // moves about a third fewer bytes than with one token tile.
@@ -444,7 +466,8 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           __syncwarp();
           if (lane == 0) mbar_arrive(&afree[slot]);
         }
-        float sq0 = 0.f, sq1 = 0.f, a0 = 0.f, a1 = 0.f;
+        uint64_t sqp = 0, ap = 0;  // packed (even, odd column) sums
+        const uint64_t kc2 = f2_pack(kC1, kC1);
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
           uint32_t ev[8];
@@ -452,14 +475,17 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           tc_wait_ld();
 #pragma unroll
           for (int j = 0; j < 8; j += 2) {
-            const float ey0 = __uint_as_float(ev[j]), ey1 = __uint_as_float(ev[j + 1]);
-            const float d0 = __uint_as_float(v[cc * 8 + j]), d1 = __uint_as_float(v[cc * 8 + j + 1]);
-            sq0 = fmaf(ey0, ex2(d0 * kC1), sq0);
-            sq1 = fmaf(ey1, ex2(d1 * kC1), sq1);
-            a0 = fmaf(ey0, d0, a0);
-            a1 = fmaf(ey1, d1, a1);
+            const uint64_t ey = f2_pack(__uint_as_float(ev[j]), __uint_as_float(ev[j + 1]));
+            const uint64_t dd = f2_pack(__uint_as_float(v[cc * 8 + j]), __uint_as_float(v[cc * 8 + j + 1]));
+            float x0, x1;
+            f2_unpack(f2_mul(dd, kc2), x0, x1);
+            sqp = f2_fma(ey, f2_pack(ex2(x0), ex2(x1)), sqp);
+            ap = f2_fma(ey, dd, ap);
           }
         }
+        float sq0, sq1, a0, a1;
+        f2_unpack(sqp, sq0, sq1);
+        f2_unpack(ap, a0, a1);
         if (last) {
           tc_fence_before();
           __syncwarp();
