@@ -199,11 +199,12 @@ UP_PROJ_13B = LayerSpec(name="llama13b_up_proj_13824x5120", m=13824, n=5120, N=C
                         x_dtype="bf16", group=128, avg_bits=2, seed=3,
                         cluster_starts=scaled_cluster_starts(5120), n_x_outliers=10)
 
-WORKLOADS = {s.name: s for s in (TINY, Q_PROJ_7B, DOWN_PROJ_7B, UP_PROJ_13B)}
-
-
 def up_proj_13b(group: int) -> LayerSpec:
+    """The 13B up_proj layer at another group size (same weights and tokens)."""
     return UP_PROJ_13B.replace(name=f"llama13b_up_proj_13824x5120_g{group}", group=group)
+
+
+WORKLOADS = {s.name: s for s in (TINY, Q_PROJ_7B, DOWN_PROJ_7B, UP_PROJ_13B, up_proj_13b(64), up_proj_13b(32))}
 
 
 # The 7B sweep: per block q,k,v,o (4096x4096), gate,up (11008 out x 4096 in), down (4096 out x 11008 in).
