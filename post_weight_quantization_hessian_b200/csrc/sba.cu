@@ -363,34 +363,45 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           ItemGeom geo;
           if (step > 0 && !dfull) geo = item_geom(p, s_order, step);
           const int nch = step == 0 ? p.nA : p.nD;
-          for (int c = 0; c < nch; ++c) {
+          // A shared-memory access by this thread waits for its MMAs to drain
+          // (about 190 cycles), so each wait is made to cover as much work as
+          // possible: right after the blocking wait on a chunk's stage, the next
+          // chunk of the same step is tested (cheap, nothing in flight) and, if
+          // its stage is full too, both chunks go out behind the one wait.
+          for (int c = 0; c < nch;) {
             if (!mbar_wait(&full[st], ph, abort_flag, p.st, 230 + st)) { ok = false; break; }
+            int st2 = st + 1;
+            uint32_t ph2 = ph;
+            if (st2 == S) { st2 = 0; ph2 ^= 1; }
+            const int take = (c + 1 < nch && mbar_test(&full[st2], ph2)) ? 2 : 1;
             tc_fence_after();
-            const uint64_t a0 = dcur, a1 = dcur + kBox16, b0 = dcur + 2 * kBox16;
-            // advancing 32 bytes along K = +2 in the descriptor's 16-byte start-address field
-            if (step == 0) {
+            for (int t = 0; t < take; ++t, ++c) {
+              const uint64_t a0 = dcur, a1 = dcur + kBox16, b0 = dcur + 2 * kBox16;
+              // advancing 32 bytes along K = +2 in the descriptor's 16-byte start-address field
+              if (step == 0) {
 #pragma unroll
-              for (int k16 = 0; k16 < 4; ++k16) {
-                const uint32_t acc = (c > 0 || k16 > 0) ? 1u : 0u;
-                tc_mma_f16(ty0, a0 + 2 * k16, b0 + 2 * k16, idesc2, acc);
-                tc_mma_f16(ty1, a1 + 2 * k16, b0 + 2 * k16, idesc2, acc);
-              }
-            } else if (dfull) {
+                for (int k16 = 0; k16 < 4; ++k16) {
+                  const uint32_t acc = (c > 0 || k16 > 0) ? 1u : 0u;
+                  tc_mma_f16(ty0, a0 + 2 * k16, b0 + 2 * k16, idesc2, acc);
+                  tc_mma_f16(ty1, a1 + 2 * k16, b0 + 2 * k16, idesc2, acc);
+                }
+              } else if (dfull) {
 #pragma unroll
-              for (int k16 = 0; k16 < 4; ++k16) {
-                tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, 1u);
-                tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, 1u);
+                for (int k16 = 0; k16 < 4; ++k16) {
+                  tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, 1u);
+                  tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, 1u);
+                }
+              } else {
+                Chunk ch;
+                chunk_at(p, geo, c, ch);
+                for (int k16 = ch.k16_lo; k16 < ch.k16_hi; ++k16) {
+                  tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, 1u);
+                  tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, 1u);
+                }
               }
-            } else {
-              Chunk ch;
-              chunk_at(p, geo, c, ch);
-              for (int k16 = ch.k16_lo; k16 < ch.k16_hi; ++k16) {
-                tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, 1u);
-                tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, 1u);
-              }
+              tc_commit(&empty[st]);
+              if (++st == S) { st = 0; ph ^= 1; dcur = d_first; } else { dcur += kStage16; }
             }
-            tc_commit(&empty[st]);
-            if (++st == S) { st = 0; ph ^= 1; dcur = d_first; } else { dcur += kStage16; }
           }
           if (!ok) break;
           tc_commit(&afull[0]);
