@@ -7,6 +7,7 @@
 #include <cstring>
 #include <string>
 #include <atomic>
+#include <vector>
 
 #include "common.cuh"
 #include "../../include/slim.h"
@@ -17,6 +18,10 @@ cudaError_t launch_hessian(const void* X, int xdtype, int64_t N, int64_t n, doub
                            int num_sms, cudaStream_t s, cudaEvent_t* kev);
 size_t hessian_ws_bytes(int64_t N, int64_t n, int xdtype);
 size_t hinv_workspace_doubles(int64_t n);
+cudaError_t launch_hessian_slices(const void* X, int64_t N, int64_t n, void* part, DevStatus* st, int num_sms,
+                                  cudaStream_t s, int slice0, int nsl);
+cudaError_t launch_hessian_reduce(int64_t N, int64_t n, const void* part, double* H, cudaStream_t s);
+int hessian_slice_tokens();
 cudaError_t launch_hinv(const double* H, int64_t n, double alpha, double* h, double* ws, DevStatus* st,
                         cudaStream_t s);
 int salience_row_blocks(int64_t m);
@@ -140,6 +145,34 @@ struct Workspace {
 
 size_t hinv_bytes(int64_t n) { return hinv_workspace_doubles(n) * sizeof(double); }
 size_t sal_bytes(int64_t m, int64_t n) { return (size_t)salience_row_blocks(m) * n * sizeof(double); }
+
+// Per host thread and device: the copy stream and events of the host-buffer
+// path (its chunked host-to-device copy of X overlaps the Hessian).
+struct HostCopy {
+  int dev = -1;
+  bool ok = false;
+  cudaStream_t cs = nullptr;
+  std::vector<cudaEvent_t> ev;
+};
+HostCopy& host_copy(int events) {
+  thread_local HostCopy hc[16];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  HostCopy& x = hc[dev & 15];
+  if (x.dev != dev) {
+    x.ok = cudaStreamCreateWithFlags(&x.cs, cudaStreamNonBlocking) == cudaSuccess;
+    x.dev = dev;
+  }
+  while (x.ok && (int)x.ev.size() < events) {
+    cudaEvent_t e;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      x.ok = false;
+      break;
+    }
+    x.ev.push_back(e);
+  }
+  return x;
+}
 
 // Layout of the full-path workspace.
 struct LayerWs {
@@ -404,6 +437,7 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
   if (rc) return rc;
   rc = check_bits(avg_bits);
   if (rc) return rc;
+  if (!(lambda >= 0.0 && lambda < 1.0) || n_tau < 1 || n_tau > 256) return SLIM_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t k = n / group;
   const size_t wb = (size_t)m * n * 4, xb = (size_t)N * n * (xdtype == SLIM_X_BF16 ? 2 : 4);
@@ -420,16 +454,82 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
   Workspace w;
   rc = w.acquire(nullptr, 0, off, s);
   if (rc) return rc;
+  const float* dW = reinterpret_cast<const float*>(w.p + o_w);
+  uint8_t* dX = w.p + o_x;
+  uint32_t* dcodes = reinterpret_cast<uint32_t*>(w.p + o_c);
+  float* dscale = reinterpret_cast<float*>(w.p + o_s);
+  float* dzero = reinterpret_cast<float*>(w.p + o_z);
+  uint8_t* dbits = w.p + o_b;
   SLIM_CUDA(cudaMemcpyAsync(w.p + o_w, W, wb, cudaMemcpyHostToDevice, s));
-  SLIM_CUDA(cudaMemcpyAsync(w.p + o_x, X, xb, cudaMemcpyHostToDevice, s));
-  rc = slim_quantize_layer(reinterpret_cast<const float*>(w.p + o_w), m, n, w.p + o_x, xdtype, N, group, avg_bits,
-                           lambda, n_tau, reinterpret_cast<uint32_t*>(w.p + o_c), reinterpret_cast<float*>(w.p + o_s),
-                           reinterpret_cast<float*>(w.p + o_z), w.p + o_b, w.p + o_ws, L.total, stream);
-  if (rc) return rc;
-  SLIM_CUDA(cudaMemcpyAsync(codes, w.p + o_c, cb, cudaMemcpyDeviceToHost, s));
-  SLIM_CUDA(cudaMemcpyAsync(scale, w.p + o_s, sb, cudaMemcpyDeviceToHost, s));
-  SLIM_CUDA(cudaMemcpyAsync(zero, w.p + o_z, sb, cudaMemcpyDeviceToHost, s));
-  SLIM_CUDA(cudaMemcpyAsync(bits, w.p + o_b, (size_t)k, cudaMemcpyDeviceToHost, s));
+  if (xdtype != SLIM_X_BF16) {
+    SLIM_CUDA(cudaMemcpyAsync(dX, X, xb, cudaMemcpyHostToDevice, s));
+    rc = slim_quantize_layer(dW, m, n, dX, xdtype, N, group, avg_bits, lambda, n_tau, dcodes, dscale, dzero, dbits,
+                             w.p + o_ws, L.total, stream);
+    if (rc) return rc;
+  } else {
+    // bf16 X: copied in chunks of whole Hessian token slices on a copy stream;
+    // each chunk's slices of H = 2 X^T X are accumulated as soon as it lands,
+    // so the tensor-core SYRK runs under the transfer. The rest of the path
+    // follows on the caller's stream.
+    int sms = 0;
+    rc = device_sms(&sms);
+    if (rc) return rc;
+    uint8_t* lw = w.p + o_ws;
+    DevStatus* st = reinterpret_cast<DevStatus*>(lw);
+    double* H = reinterpret_cast<double*>(lw + L.off_H);
+    double* h = reinterpret_cast<double*>(lw + L.off_h);
+    double* S = reinterpret_cast<double*>(lw + L.off_S);
+    int32_t* order = reinterpret_cast<int32_t*>(lw + L.off_order);
+    double* kl = reinterpret_cast<double*>(lw + L.off_kl);
+    int32_t* pstar = reinterpret_cast<int32_t*>(lw + L.off_pstar);
+    uint8_t* scratch = lw + L.off_scratch;
+    const int64_t stok = hessian_slice_tokens();
+    const int nsl = (int)((N + stok - 1) / stok);
+    const int per = (nsl + 63) / 64;               // slices per chunk: at most 64 chunks
+    const int nch = (nsl + per - 1) / per;
+    HostCopy& hc = host_copy(nch + 1);
+    if (!hc.ok) return SLIM_ECUDA;
+    SLIM_CUDA(cudaMemsetAsync(st, 0, kStatusBytes, s));
+    SLIM_CUDA(cudaEventRecord(hc.ev[nch], s));          // the workspace exists before the copies start
+    SLIM_CUDA(cudaStreamWaitEvent(hc.cs, hc.ev[nch], 0));
+    const size_t row_bytes = (size_t)n * 2;
+    // on every return from here, the caller's stream first waits for the last
+    // copy, so the workspace is never released under a copy still in flight
+    struct CopyJoin {
+      cudaStream_t s;
+      cudaEvent_t e;
+      ~CopyJoin() { cudaStreamWaitEvent(s, e, 0); }
+    } join{s, hc.ev[nch - 1]};
+    for (int c = 0; c < nch; ++c) {
+      const int64_t r0 = (int64_t)c * per * stok;
+      const int64_t r1 = (r0 + (int64_t)per * stok < N) ? r0 + (int64_t)per * stok : N;
+      SLIM_CUDA(cudaMemcpyAsync(dX + r0 * row_bytes, static_cast<const uint8_t*>(X) + r0 * row_bytes,
+                                (size_t)(r1 - r0) * row_bytes, cudaMemcpyHostToDevice, hc.cs));
+      SLIM_CUDA(cudaEventRecord(hc.ev[c], hc.cs));
+    }
+    if (injected("hessian")) return SLIM_EINJECTED;
+    for (int c = 0; c < nch; ++c) {
+      SLIM_CUDA(cudaStreamWaitEvent(s, hc.ev[c], 0));
+      const int s0 = c * per, cnt = (s0 + per < nsl) ? per : nsl - s0;
+      SLIM_CUDA(launch_hessian_slices(dX, N, n, scratch, st, sms, s, s0, cnt));
+    }
+    SLIM_CUDA(launch_hessian_reduce(N, n, scratch, H, s));
+    if (injected("hinv_diag")) return SLIM_EINJECTED;
+    SLIM_CUDA(launch_hinv(H, n, kDampAlpha, h, reinterpret_cast<double*>(scratch), st, s));
+    if (injected("salience")) return SLIM_EINJECTED;
+    SLIM_CUDA(launch_salience(dW, m, n, h, group, S, order, reinterpret_cast<double*>(scratch), s));
+    if (injected("sba_search")) return SLIM_EINJECTED;
+    SLIM_CUDA(launch_sba(dW, m, n, dX, xdtype, N, group, avg_bits, order, kl, pstar, dbits, scratch, st, sms, s,
+                         nullptr));
+    if (injected("sqc")) return SLIM_EINJECTED;
+    SLIM_CUDA(launch_sqc(dW, m, n, h, dbits, group, avg_bits, lambda, n_tau, dcodes, dscale, dzero, nullptr, sms, s));
+    rc = finish(s, st);
+    if (rc) return rc;
+  }
+  SLIM_CUDA(cudaMemcpyAsync(codes, dcodes, cb, cudaMemcpyDeviceToHost, s));
+  SLIM_CUDA(cudaMemcpyAsync(scale, dscale, sb, cudaMemcpyDeviceToHost, s));
+  SLIM_CUDA(cudaMemcpyAsync(zero, dzero, sb, cudaMemcpyDeviceToHost, s));
+  SLIM_CUDA(cudaMemcpyAsync(bits, dbits, (size_t)k, cudaMemcpyDeviceToHost, s));
   SLIM_CUDA(cudaStreamSynchronize(s));
   return SLIM_OK;
 }

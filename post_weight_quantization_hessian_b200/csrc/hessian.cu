@@ -38,6 +38,7 @@ constexpr int HS_SMEM = HS_STAGES * HS_STAGE + 1024 /*align*/ + 256 /*barriers*/
 struct SyrkParams {
   int64_t N, n;
   int nblk, npairs, nslices;
+  int slice0, launch_slices;  // this launch covers slices [slice0, slice0 + launch_slices)
   int64_t slice_tokens;  // multiple of 64
   float* part;           // [nslices][npairs][256][256]
   DevStatus* st;
@@ -76,13 +77,13 @@ __global__ void __launch_bounds__(192, 1) syrk_tc_kernel(const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tslot;
-  const int units = p.npairs * p.nslices;
+  const int units = p.npairs * p.launch_slices;
 
   if (warp == 0) {
     if (lane == 0) {
       uint32_t it = 0;
       for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
-        const int slice = u / p.npairs, pair = u - slice * p.npairs;
+        const int sl = u / p.npairs, pair = u - sl * p.npairs, slice = p.slice0 + sl;
         int bb, ba;
         tri_decode(pair, bb, ba);
         const int64_t t0 = (int64_t)slice * p.slice_tokens;
@@ -115,7 +116,7 @@ __global__ void __launch_bounds__(192, 1) syrk_tc_kernel(const __grid_constant__
       uint32_t it = 0, ui = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
-        const int slice = u / p.npairs, pair = u - slice * p.npairs;
+        const int sl = u / p.npairs, pair = u - sl * p.npairs, slice = p.slice0 + sl;
         int bb, ba;
         tri_decode(pair, bb, ba);
         const int64_t t0 = (int64_t)slice * p.slice_tokens;
@@ -154,7 +155,7 @@ __global__ void __launch_bounds__(192, 1) syrk_tc_kernel(const __grid_constant__
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++ui) {
       if (!mbar_wait(tfull, ui & 1, abort_flag, p.st, 150)) break;
       tc_fence_after();
-      float* dst = p.part + (size_t)u * HS_TILE * HS_TILE;
+      float* dst = p.part + ((size_t)p.slice0 * p.npairs + u) * HS_TILE * HS_TILE;
 #pragma unroll 1
       for (int q = 0; q < 2; ++q) {
         const int row = q * 128 + wq * 32 + lane;
@@ -287,6 +288,41 @@ size_t hessian_ws_bytes(int64_t N, int64_t n, int xdtype) {
   return xdtype == 1 ? syrk_plan_bf16(N, n).part_bytes : syrk_plan_f32(N, n).part_bytes;
 }
 
+// bf16 X, token slices [slice0, slice0 + nsl) only: their fp32 partials. The
+// rows of those slices must be in X; other rows are not read.
+cudaError_t launch_hessian_slices(const void* X, int64_t N, int64_t n, void* part, DevStatus* st, int num_sms,
+                                  cudaStream_t s, int slice0, int nsl) {
+  const SyrkPlan pl = syrk_plan_bf16(N, n);
+  CUtensorMap tm;
+  if (!make_tmap_bf16(&tm, X, (uint64_t)n, (uint64_t)N, 64, 64)) return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(syrk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  SyrkParams p;
+  p.N = N; p.n = n; p.nblk = pl.nblk; p.npairs = pl.npairs; p.nslices = pl.nslices;
+  p.slice0 = slice0; p.launch_slices = nsl;
+  p.slice_tokens = pl.slice_tokens; p.part = static_cast<float*>(part); p.st = st;
+  const int units = pl.npairs * nsl;
+  const int grid = units < num_sms ? units : num_sms;
+  syrk_tc_kernel<<<grid, 192, HS_SMEM, s>>>(tm, p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// H from the fp32 partials of all slices (bf16 X).
+cudaError_t launch_hessian_reduce(int64_t N, int64_t n, const void* part, double* H, cudaStream_t s) {
+  const SyrkPlan pl = syrk_plan_bf16(N, n);
+  syrk_reduce_kernel<<<dim3(HS_TILE * HS_TILE / 256, pl.npairs), 256, 0, s>>>(static_cast<const float*>(part),
+                                                                              pl.npairs, pl.nslices, n, H);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+int hessian_slice_tokens() { return (int)kSyrkSliceTokens; }
+
 cudaError_t launch_hessian(const void* X, int xdtype, int64_t N, int64_t n, double* H, void* part, DevStatus* st,
                            int num_sms, cudaStream_t s, cudaEvent_t* kev) {
   if (xdtype == 1) {
@@ -301,6 +337,7 @@ cudaError_t launch_hessian(const void* X, int xdtype, int64_t N, int64_t n, doub
     }
     SyrkParams p;
     p.N = N; p.n = n; p.nblk = pl.nblk; p.npairs = pl.npairs; p.nslices = pl.nslices;
+    p.slice0 = 0; p.launch_slices = pl.nslices;
     p.slice_tokens = pl.slice_tokens; p.part = static_cast<float*>(part); p.st = st;
     const int units = pl.npairs * pl.nslices;
     const int grid = units < num_sms ? units : num_sms;

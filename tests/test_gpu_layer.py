@@ -65,6 +65,24 @@ def test_small_layer_bf16(kw):
     run_and_compare(syn.LayerSpec(**base), h_rtol=1e-3)
 
 
+@pytest.mark.parametrize("x_dtype", ["bf16", "f32"])
+def test_host_buffers_match_device_path(x_dtype):
+    """slim_quantize_layer_host (host arrays in and out; bf16 X copied in chunks of
+    whole Hessian slices whose SYRK runs as each lands) gives the device path's
+    outputs bit for bit. N spans three 16384-token slices and a ragged tail."""
+    spec = syn.LayerSpec(name="host_path", m=256, n=512, N=3 * 16384 + 1808, x_dtype=x_dtype, group=128,
+                         avg_bits=2, seed=11, n_w_salient=6, w_scale=6.0, n_x_outliers=3, x_scale=25.0)
+    W, Xh, Wd, Xd = device_inputs(spec)
+    d = slim.slim_quantize_layer_ex(Wd, Xd, spec.group, spec.avg_bits, spec.lam, spec.n_tau, want_H=False)
+    Xn = Xh.view(np.uint16) if x_dtype == "bf16" else Xh
+    codes, scale, zero, bits = slim.slim_quantize_layer_host(W, np.ascontiguousarray(Xn), spec.group, spec.avg_bits,
+                                                             spec.lam, spec.n_tau)
+    assert np.array_equal(codes.view(np.uint32), d["codes"].cpu().numpy().view(np.uint32))
+    assert np.array_equal(scale, d["scale"].cpu().numpy())
+    assert np.array_equal(zero, d["zero"].cpu().numpy())
+    assert np.array_equal(bits, d["bits"].cpu().numpy())
+
+
 FULL_SIZE = [w for w in ("llama7b_q_proj_4096x4096", "llama7b_down_proj_4096x11008", "llama13b_up_proj_13824x5120",
                           "llama13b_up_proj_13824x5120_g64", "llama13b_up_proj_13824x5120_g32")
              if os.path.exists(os.path.join(os.path.dirname(__file__), "golden", f"{w}.json"))]
