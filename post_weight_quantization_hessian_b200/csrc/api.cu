@@ -28,6 +28,15 @@ int salience_row_blocks(int64_t m);
 cudaError_t launch_salience(const float* W, int64_t m, int64_t n, const double* h, int group, double* S,
                             int32_t* order, double* part, cudaStream_t st);
 size_t sba_ws_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group);
+size_t sba_prep_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group);
+size_t sba_search_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group);
+cudaError_t launch_sba_prep_w(const float* W, int64_t m, int64_t n, int64_t N, int xdtype, int group, int avg_bits,
+                              uint8_t* pw, DevStatus* st, int num_sms, int bps, cudaStream_t s);
+cudaError_t launch_sba_prep_x(const void* X, int64_t m, int64_t n, int64_t N, int xdtype, int group, int64_t t0,
+                              int64_t t1, uint8_t* pw, DevStatus* st, int num_sms, int bps, cudaStream_t s);
+cudaError_t launch_sba_search(int64_t m, int64_t n, int xdtype, int64_t N, int group, int avg_bits,
+                              const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, const uint8_t* pw,
+                              uint8_t* sw, DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev);
 cudaError_t launch_sba(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
                        int avg_bits, const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, uint8_t* ws,
                        DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev);
@@ -146,12 +155,17 @@ struct Workspace {
 size_t hinv_bytes(int64_t n) { return hinv_workspace_doubles(n) * sizeof(double); }
 size_t sal_bytes(int64_t m, int64_t n) { return (size_t)salience_row_blocks(m) * n * sizeof(double); }
 
-// Per host thread and device: the copy stream and events of the host-buffer
-// path (its chunked host-to-device copy of X overlaps the Hessian).
+// Per host thread and device: the side streams of the whole-layer paths.
+// cs carries the host-buffer path's chunked host-to-device copy of X (it
+// overlaps the Hessian; ev are its events); ps, at the lowest priority,
+// prepares the SBA operands beside other stages (pe[0] forks it, pe[1] joins
+// it): beside the chunked Hessian in the host-buffer path, beside the
+// latency-bound inverse-Hessian stage in the device path.
 struct HostCopy {
   int dev = -1;
   bool ok = false;
-  cudaStream_t cs = nullptr;
+  cudaStream_t cs = nullptr, ps = nullptr;
+  cudaEvent_t pe[2] = {};
   std::vector<cudaEvent_t> ev;
 };
 HostCopy& host_copy(int events) {
@@ -160,7 +174,12 @@ HostCopy& host_copy(int events) {
   cudaGetDevice(&dev);
   HostCopy& x = hc[dev & 15];
   if (x.dev != dev) {
-    x.ok = cudaStreamCreateWithFlags(&x.cs, cudaStreamNonBlocking) == cudaSuccess;
+    int least = 0, greatest = 0;
+    cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    x.ok = cudaStreamCreateWithFlags(&x.cs, cudaStreamNonBlocking) == cudaSuccess &&
+           cudaStreamCreateWithPriority(&x.ps, cudaStreamNonBlocking, least) == cudaSuccess &&
+           cudaEventCreateWithFlags(&x.pe[0], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&x.pe[1], cudaEventDisableTiming) == cudaSuccess;
     x.dev = dev;
   }
   while (x.ok && (int)x.ev.size() < events) {
@@ -174,9 +193,12 @@ HostCopy& host_copy(int events) {
   return x;
 }
 
-// Layout of the full-path workspace.
+// Layout of the full-path workspace. The scratch region holds the SBA
+// operands, prepared beside the Hessian (at off_scratch), and behind them
+// (off_rest) the scratch that the Hessian's partial sums, hinv, salience and
+// the SBA search use in turn.
 struct LayerWs {
-  size_t off_H, off_h, off_S, off_order, off_kl, off_pstar, off_scratch, total;
+  size_t off_H, off_h, off_S, off_order, off_kl, off_pstar, off_scratch, off_rest, total;
 };
 LayerWs layer_ws(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
   LayerWs w{};
@@ -189,13 +211,44 @@ LayerWs layer_ws(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
   w.off_order = off; off = al256(off + (size_t)k * 4);
   w.off_kl = off; off = al256(off + (size_t)P * 8);
   w.off_pstar = off; off = al256(off + 8);
-  size_t scratch = hessian_ws_bytes(N, n, xdtype);
-  size_t t = hinv_bytes(n); if (t > scratch) scratch = t;
-  t = sal_bytes(m, n); if (t > scratch) scratch = t;
-  t = sba_ws_bytes(m, n, N, xdtype, group); if (t > scratch) scratch = t;
-  w.off_scratch = off; off = al256(off + scratch);
+  size_t rest = hinv_bytes(n);
+  size_t t = sal_bytes(m, n); if (t > rest) rest = t;
+  t = sba_search_bytes(m, n, N, xdtype, group); if (t > rest) rest = t;
+  t = hessian_ws_bytes(N, n, xdtype); if (t > rest) rest = t;
+  const size_t prep = al256(sba_prep_bytes(m, n, N, xdtype, group));
+  w.off_scratch = off;
+  w.off_rest = off + prep;
+  off = al256(off + prep + rest);
   w.total = off;
   return w;
+}
+
+// On every return, s first waits for all work queued so far on the side
+// stream `from` (through event e), so a workspace released or reused in s's
+// order is never touched by work still running there.
+struct JoinOnExit {
+  cudaStream_t s, from;
+  cudaEvent_t e;
+  ~JoinOnExit() {
+    if (cudaEventRecord(e, from) == cudaSuccess) cudaStreamWaitEvent(s, e, 0);
+  }
+};
+
+// Forks onto the side stream, once everything queued on s so far is done,
+// the preparation of the SBA weight operands and (X non-null) of all of X,
+// at bps blocks per SM. Join with join_prepare.
+cudaError_t fork_prepare(HostCopy& side, const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N,
+                         int group, int avg_bits, uint8_t* pw, DevStatus* st, int sms, int bps, cudaStream_t s) {
+  cudaError_t e = cudaEventRecord(side.pe[0], s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(side.ps, side.pe[0], 0);
+  if (e == cudaSuccess) e = launch_sba_prep_w(W, m, n, N, xdtype, group, avg_bits, pw, st, sms, bps, side.ps);
+  if (e == cudaSuccess && X) e = launch_sba_prep_x(X, m, n, N, xdtype, group, 0, N, pw, st, sms, bps, side.ps);
+  return e;
+}
+cudaError_t join_prepare(HostCopy& side, cudaStream_t s) {
+  cudaError_t e = cudaEventRecord(side.pe[1], side.ps);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, side.pe[1], 0);
+  return e;
 }
 
 }  // namespace
@@ -376,6 +429,10 @@ int slim_quantize_layer_ex(const float* W, int64_t m, int64_t n, const void* X, 
   int32_t* pstar = reinterpret_cast<int32_t*>(w.p + L.off_pstar);
   uint8_t* tau = diag ? diag->tau_idx : nullptr;
   uint8_t* scratch = w.p + L.off_scratch;
+  uint8_t* rest = w.p + L.off_rest;
+  HostCopy& side = host_copy(0);
+  if (!side.ok) return SLIM_ECUDA;
+  JoinOnExit join{s, side.ps, side.pe[1]};
 
   cudaEvent_t ev[10] = {};
   const bool timed = diag != nullptr;
@@ -388,16 +445,21 @@ int slim_quantize_layer_ex(const float* W, int64_t m, int64_t n, const void* X, 
     SLIM_CUDA(cudaMemsetAsync(st, 0, kStatusBytes, s));
     rec(0);
     if (injected("hessian")) return SLIM_EINJECTED;
-    SLIM_CUDA(launch_hessian(X, xdtype, N, n, H, scratch, st, sms, s, kev_h));
+    SLIM_CUDA(launch_hessian(X, xdtype, N, n, H, rest, st, sms, s, kev_h));
     rec(1);
+    // beside the latency-bound inverse: one block per SM leaves each SM the
+    // registers and shared memory of one factorization CTA plus the updates
+    SLIM_CUDA(fork_prepare(side, W, m, n, X, xdtype, N, group, avg_bits, scratch, st, sms, 1, s));
     if (injected("hinv_diag")) return SLIM_EINJECTED;
-    SLIM_CUDA(launch_hinv(H, n, kDampAlpha, h, reinterpret_cast<double*>(scratch), st, s));
+    SLIM_CUDA(launch_hinv(H, n, kDampAlpha, h, reinterpret_cast<double*>(rest), st, s));
     rec(2);
     if (injected("salience")) return SLIM_EINJECTED;
-    SLIM_CUDA(launch_salience(W, m, n, h, group, S, order, reinterpret_cast<double*>(scratch), s));
+    SLIM_CUDA(launch_salience(W, m, n, h, group, S, order, reinterpret_cast<double*>(rest), s));
     rec(3);
     if (injected("sba_search")) return SLIM_EINJECTED;
-    SLIM_CUDA(launch_sba(W, m, n, X, xdtype, N, group, avg_bits, order, kl, pstar, bits, scratch, st, sms, s, kev_s));
+    SLIM_CUDA(join_prepare(side, s));
+    SLIM_CUDA(launch_sba_search(m, n, xdtype, N, group, avg_bits, order, kl, pstar, bits, scratch, rest, st, sms, s,
+                                kev_s));
     rec(4);
     if (injected("sqc")) return SLIM_EINJECTED;
     SLIM_CUDA(launch_sqc(W, m, n, h, bits, group, avg_bits, lambda, n_tau, codes, scale, zero, tau, sms, s));
@@ -483,6 +545,7 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
     double* kl = reinterpret_cast<double*>(lw + L.off_kl);
     int32_t* pstar = reinterpret_cast<int32_t*>(lw + L.off_pstar);
     uint8_t* scratch = lw + L.off_scratch;
+    uint8_t* rest = lw + L.off_rest;
     const int64_t stok = hessian_slice_tokens();
     const int nsl = (int)((N + stok - 1) / stok);
     const int per = (nsl + 63) / 64;               // slices per chunk: at most 64 chunks
@@ -493,13 +556,10 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
     SLIM_CUDA(cudaEventRecord(hc.ev[nch], s));          // the workspace exists before the copies start
     SLIM_CUDA(cudaStreamWaitEvent(hc.cs, hc.ev[nch], 0));
     const size_t row_bytes = (size_t)n * 2;
-    // on every return from here, the caller's stream first waits for the last
-    // copy, so the workspace is never released under a copy still in flight
-    struct CopyJoin {
-      cudaStream_t s;
-      cudaEvent_t e;
-      ~CopyJoin() { cudaStreamWaitEvent(s, e, 0); }
-    } join{s, hc.ev[nch - 1]};
+    // on every return from here, the caller's stream first waits for the
+    // copies and the operand preparation, so the workspace is never released
+    // under work still in flight
+    JoinOnExit join{s, hc.cs, hc.ev[nch]}, join_prep{s, hc.ps, hc.pe[1]};
     for (int c = 0; c < nch; ++c) {
       const int64_t r0 = (int64_t)c * per * stok;
       const int64_t r1 = (r0 + (int64_t)per * stok < N) ? r0 + (int64_t)per * stok : N;
@@ -507,20 +567,28 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
                                 (size_t)(r1 - r0) * row_bytes, cudaMemcpyHostToDevice, hc.cs));
       SLIM_CUDA(cudaEventRecord(hc.ev[c], hc.cs));
     }
+    // W (copied on s above) is resident: its operands are prepared on the
+    // side stream, then each chunk of X is converted there as it lands
+    SLIM_CUDA(fork_prepare(hc, dW, m, n, nullptr, xdtype, N, group, avg_bits, scratch, st, sms, 2, s));
     if (injected("hessian")) return SLIM_EINJECTED;
     for (int c = 0; c < nch; ++c) {
+      const int64_t r0 = (int64_t)c * per * stok;
+      const int64_t r1 = (r0 + (int64_t)per * stok < N) ? r0 + (int64_t)per * stok : N;
       SLIM_CUDA(cudaStreamWaitEvent(s, hc.ev[c], 0));
       const int s0 = c * per, cnt = (s0 + per < nsl) ? per : nsl - s0;
-      SLIM_CUDA(launch_hessian_slices(dX, N, n, scratch, st, sms, s, s0, cnt));
+      SLIM_CUDA(launch_hessian_slices(dX, N, n, rest, st, sms, s, s0, cnt));
+      SLIM_CUDA(cudaStreamWaitEvent(hc.ps, hc.ev[c], 0));
+      SLIM_CUDA(launch_sba_prep_x(dX, m, n, N, xdtype, group, r0, r1, scratch, st, sms, 2, hc.ps));
     }
-    SLIM_CUDA(launch_hessian_reduce(N, n, scratch, H, s));
+    SLIM_CUDA(launch_hessian_reduce(N, n, rest, H, s));
     if (injected("hinv_diag")) return SLIM_EINJECTED;
-    SLIM_CUDA(launch_hinv(H, n, kDampAlpha, h, reinterpret_cast<double*>(scratch), st, s));
+    SLIM_CUDA(launch_hinv(H, n, kDampAlpha, h, reinterpret_cast<double*>(rest), st, s));
     if (injected("salience")) return SLIM_EINJECTED;
-    SLIM_CUDA(launch_salience(dW, m, n, h, group, S, order, reinterpret_cast<double*>(scratch), s));
+    SLIM_CUDA(launch_salience(dW, m, n, h, group, S, order, reinterpret_cast<double*>(rest), s));
     if (injected("sba_search")) return SLIM_EINJECTED;
-    SLIM_CUDA(launch_sba(dW, m, n, dX, xdtype, N, group, avg_bits, order, kl, pstar, dbits, scratch, st, sms, s,
-                         nullptr));
+    SLIM_CUDA(join_prepare(hc, s));
+    SLIM_CUDA(launch_sba_search(m, n, xdtype, N, group, avg_bits, order, kl, pstar, dbits, scratch, rest, st, sms, s,
+                                nullptr));
     if (injected("sqc")) return SLIM_EINJECTED;
     SLIM_CUDA(launch_sqc(dW, m, n, h, dbits, group, avg_bits, lambda, n_tau, dcodes, dscale, dzero, nullptr, sms, s));
     rc = finish(s, st);

@@ -10,8 +10,9 @@
 //
 //   Cholesky, right-looking, per diagonal block K:
 //     pp(K)     every CTA applies step K-1's update to block K and factors it
-//               (L_KK, M_KK = L_KK^-1); CTA 0 stores them, CTA b > 0 updates
+//               (L_KK, M_KK = L_KK^-1); CTA 0 stores M_KK, CTA b > 0 updates
 //               its block row I = K + b of column K and stores L_IK = A_IK M_KK^T
+//               (A_KK itself is never overwritten: every CTA reads it)
 //     trail(K)  A_IJ -= L_IK L_JK^T for K + 2 <= J <= I
 //   Inverse, forward substitution of L M = I, right-looking, per block row I:
 //     rowmult(I)    M_IJ = M_II R_IJ for J < I (R accumulates -sum L_IK M_KJ)
@@ -522,10 +523,13 @@ __global__ void __launch_bounds__(HT, 1) pp_kernel(double* __restrict__ A, doubl
     __syncthreads();
     panel_tri(D, Mi, nbk, aIK, n, nbi, nbk);
   } else {
+    // Only M_KK goes out. L_KK stays in shared memory: no later kernel reads
+    // a diagonal block of L, and writing it over A_KK here would race with
+    // the CTAs of this launch that have not yet loaded A_KK (nothing makes
+    // them resident at once).
     double* mKK = M + (int64_t)K * NB * n + (int64_t)K * NB;
     for (int e = threadIdx.x; e < nbk * nbk; e += HT) {
       const int r = e / nbk, c = e - r * nbk;
-      aKK[(int64_t)r * n + c] = (c <= r) ? D[r * LD + c] : 0.0;
       mKK[(int64_t)r * n + c] = (c <= r) ? Mi[r * LD + c] : 0.0;
     }
   }

@@ -112,23 +112,35 @@ __global__ void __launch_bounds__(256) sba_prep_kernel(const float* __restrict__
   }
 }
 
-// bf16 -> fp16, 8 elements per thread (16-byte loads and stores).
-__global__ void x_to_f16_kernel(const uint4* __restrict__ X, int64_t n8, uint4* __restrict__ Y, DevStatus* st) {
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n8; e += (int64_t)gridDim.x * blockDim.x) {
-    const uint4 v = X[e];
-    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-    uint32_t out[4];
-    bool bad = false;
+// bf16 -> fp16, 8 elements per 16-byte load and store; XU loads in flight
+// per thread, so that a grid of a few blocks per SM still keeps enough bytes
+// in flight to stream at HBM rate.
+constexpr int XU = 8;
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 v, bool& bad) {
+  const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float a = __uint_as_float(in[q] << 16), b = __uint_as_float(in[q] & 0xFFFF0000u);
-      bad |= !(fabsf(a) <= kHalfMax) || !(fabsf(b) <= kHalfMax);
-      const __half2 h = __floats2half2_rn(a, b);
-      out[q] = *reinterpret_cast<const uint32_t*>(&h);
-    }
-    if (bad) record_failure(st, kStatusRange, 310);
-    Y[e] = make_uint4(out[0], out[1], out[2], out[3]);
+  for (int q = 0; q < 4; ++q) {
+    const float a = __uint_as_float(in[q] << 16), b = __uint_as_float(in[q] & 0xFFFF0000u);
+    bad |= !(fabsf(a) <= kHalfMax) || !(fabsf(b) <= kHalfMax);
+    const __half2 h = __floats2half2_rn(a, b);
+    out[q] = *reinterpret_cast<const uint32_t*>(&h);
   }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+__global__ void x_to_f16_kernel(const uint4* __restrict__ X, int64_t n8, uint4* __restrict__ Y, DevStatus* st) {
+  const int64_t T = (int64_t)gridDim.x * blockDim.x;
+  bool bad = false;
+  int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; e + (XU - 1) * T < n8; e += XU * T) {
+    uint4 v[XU];
+#pragma unroll
+    for (int u = 0; u < XU; ++u) v[u] = X[e + u * T];
+#pragma unroll
+    for (int u = 0; u < XU; ++u) Y[e + u * T] = bf16x8_to_f16x8(v[u], bad);
+  }
+  for (; e < n8; e += T) Y[e] = bf16x8_to_f16x8(X[e], bad);
+  if (bad) record_failure(st, kStatusRange, 310);
 }
 
 __global__ void x_split_kernel(const float* __restrict__ X, int64_t N, int64_t n, __half* __restrict__ Xc,
@@ -596,6 +608,8 @@ __global__ void sba_final_kernel(const double* __restrict__ kl_part, int n_tt, i
 }
 
 // ---------------------------------------------------------------- host side
+// Workspace: [prepared operands: Wb, E0, Dp, Dm, X as fp16][search: partials, KL parts].
+// The prepared region depends only on W and X, so it can be filled early.
 struct SbaPlan {
   int k, P, ksplit, n_tt, n_tp, n_ot, stages, nA, nD;
   size_t off_wb, off_e0, off_dp, off_dm, off_xc, off_part, off_klp, total;
@@ -638,34 +652,72 @@ SbaPlan sba_plan(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
 size_t sba_ws_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
   return sba_plan(m, n, N, xdtype, group).total;
 }
+size_t sba_prep_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
+  return sba_plan(m, n, N, xdtype, group).off_part;
+}
+size_t sba_search_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
+  const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
+  return pl.total - pl.off_part;
+}
 
-cudaError_t launch_sba(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
-                       int avg_bits, const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, uint8_t* ws,
-                       DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev) {
+// The weight-side fp16 operands (RTN at b-1, b, b+1) into the prepared region
+// (pw: sba_prep_bytes). bps caps the resident blocks per SM: a small cap
+// leaves room on every SM for kernels that run beside these grid-stride loops
+// on other streams.
+cudaError_t launch_sba_prep_w(const float* W, int64_t m, int64_t n, int64_t N, int xdtype, int group, int avg_bits,
+                              uint8_t* pw, DevStatus* st, int num_sms, int bps, cudaStream_t s) {
   const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
   if (pl.k > SB_MAX_K) return cudaErrorInvalidValue;
-  __half* Wb = reinterpret_cast<__half*>(ws + pl.off_wb);
-  __half* E0 = reinterpret_cast<__half*>(ws + pl.off_e0);
-  __half* Dp = reinterpret_cast<__half*>(ws + pl.off_dp);
-  __half* Dm = reinterpret_cast<__half*>(ws + pl.off_dm);
-  __half* Xc = reinterpret_cast<__half*>(ws + pl.off_xc);
-  float* part = reinterpret_cast<float*>(ws + pl.off_part);
-  double* klp = reinterpret_cast<double*>(ws + pl.off_klp);
-
+  __half* Wb = reinterpret_cast<__half*>(pw + pl.off_wb);
+  __half* E0 = reinterpret_cast<__half*>(pw + pl.off_e0);
+  __half* Dp = reinterpret_cast<__half*>(pw + pl.off_dp);
+  __half* Dm = reinterpret_cast<__half*>(pw + pl.off_dm);
   const int64_t pairs = m * pl.k;
   int pgrid = (int)((pairs + 7) / 8);
-  if (pgrid > num_sms * 16) pgrid = num_sms * 16;
+  if (pgrid > num_sms * 2 * bps) pgrid = num_sms * 2 * bps;
   switch (group) {
     case 32: sba_prep_kernel<32><<<pgrid, 256, 0, s>>>(W, m, n, avg_bits, Wb, E0, Dp, Dm, st); break;
     case 64: sba_prep_kernel<64><<<pgrid, 256, 0, s>>>(W, m, n, avg_bits, Wb, E0, Dp, Dm, st); break;
     case 128: sba_prep_kernel<128><<<pgrid, 256, 0, s>>>(W, m, n, avg_bits, Wb, E0, Dp, Dm, st); break;
     default: return cudaErrorInvalidValue;
   }
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// Rows [t0, t1) of X as fp16 operands (bf16: converted; fp32: split into a
+// high and a low fp16 part) into the prepared region.
+cudaError_t launch_sba_prep_x(const void* X, int64_t m, int64_t n, int64_t N, int xdtype, int group, int64_t t0,
+                              int64_t t1, uint8_t* pw, DevStatus* st, int num_sms, int bps, cudaStream_t s) {
+  const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
+  if (t0 < 0 || t1 > N || t1 < t0) return cudaErrorInvalidValue;
+  if (t1 == t0) return cudaSuccess;
+  __half* Xc = reinterpret_cast<__half*>(pw + pl.off_xc);
   if (pl.ksplit == 2) {
-    x_split_kernel<<<num_sms * 8, 256, 0, s>>>(static_cast<const float*>(X), N, n, Xc, st);
+    x_split_kernel<<<num_sms * bps, 256, 0, s>>>(static_cast<const float*>(X) + t0 * n, t1 - t0, n,
+                                                 Xc + t0 * 2 * n, st);
   } else {
-    x_to_f16_kernel<<<num_sms * 8, 256, 0, s>>>(static_cast<const uint4*>(X), N * n / 8, reinterpret_cast<uint4*>(Xc), st);
+    x_to_f16_kernel<<<num_sms * bps, 256, 0, s>>>(static_cast<const uint4*>(X) + t0 * n / 8, (t1 - t0) * n / 8,
+                                                  reinterpret_cast<uint4*>(Xc + t0 * n), st);
   }
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// Scoring, merge and final selection on the prepared operands (pw) with the
+// search region (sw: sba_search_bytes) for the partial sums.
+cudaError_t launch_sba_search(int64_t m, int64_t n, int xdtype, int64_t N, int group, int avg_bits,
+                              const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, const uint8_t* pw,
+                              uint8_t* sw, DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev) {
+  const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
+  if (pl.k > SB_MAX_K) return cudaErrorInvalidValue;
+  const __half* Wb = reinterpret_cast<const __half*>(pw + pl.off_wb);
+  const __half* E0 = reinterpret_cast<const __half*>(pw + pl.off_e0);
+  const __half* Dp = reinterpret_cast<const __half*>(pw + pl.off_dp);
+  const __half* Dm = reinterpret_cast<const __half*>(pw + pl.off_dm);
+  const __half* Xc = reinterpret_cast<const __half*>(pw + pl.off_xc);
+  float* part = reinterpret_cast<float*>(sw);
+  double* klp = reinterpret_cast<double*>(sw + (pl.off_klp - pl.off_part));
   const void* xptr = Xc;
   SbaTmaps tm;
   bool ok = make_tmap_f16(&tm.x, xptr, (uint64_t)(n * pl.ksplit), (uint64_t)N, SB_BK, SB_BM);
@@ -693,8 +745,19 @@ cudaError_t launch_sba(const float* W, int64_t m, int64_t n, const void* X, int 
   }
   sba_merge_kernel<<<pl.n_tt, SB_BM, msmem, s>>>(part, pl.n_ot, pl.P, N, pl.n_tt, klp);
   sba_final_kernel<<<1, 256, 0, s>>>(klp, pl.n_tt, pl.P, N, order, pl.k, avg_bits, kl, p_star, bits);
-  count_launches(5);
+  count_launches(3);
   return cudaGetLastError();
+}
+
+cudaError_t launch_sba(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
+                       int avg_bits, const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, uint8_t* ws,
+                       DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev) {
+  const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
+  cudaError_t e = launch_sba_prep_w(W, m, n, N, xdtype, group, avg_bits, ws, st, num_sms, 8, s);
+  if (e == cudaSuccess) e = launch_sba_prep_x(X, m, n, N, xdtype, group, 0, N, ws, st, num_sms, 8, s);
+  if (e != cudaSuccess) return e;
+  return launch_sba_search(m, n, xdtype, N, group, avg_bits, order, kl, p_star, bits, ws, ws + pl.off_part, st,
+                           num_sms, s, kev);
 }
 
 }  // namespace slim

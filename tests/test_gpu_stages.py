@@ -54,6 +54,32 @@ def test_hinv_diag(n):
     np.testing.assert_allclose(h, O.hinv_diag(H, 0.01), rtol=1e-9)
 
 
+def test_hinv_diag_beside_a_busy_gpu():
+    """The factorization must not depend on its CTAs being resident together.
+
+    GEMMs on another stream hold most SMs' shared memory while the inverse is
+    computed, so the CTAs of one launch start at different times; a CTA that
+    wrote a block other CTAs of its launch still had to read would show here.
+    """
+    n = 2048
+    rng = np.random.default_rng(7)
+    X = rng.standard_normal((2 * n, n))
+    X[:, 11] *= 30.0
+    H = O.hessian(X)
+    ref = O.hinv_diag(H, 0.01)
+    Hd = torch.from_numpy(H).cuda()
+    a = torch.randn(8192, 8192, dtype=torch.bfloat16, device="cuda")
+    busy, work = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        with torch.cuda.stream(busy):
+            for _ in range(24):
+                a = (a @ a).clamp_(-1.0, 1.0)
+        h = slim.slim_hinv_diag(Hd, 0.01, stream=work).cpu().numpy()
+        np.testing.assert_allclose(h, ref, rtol=1e-9)
+    torch.cuda.synchronize()
+
+
 def test_hinv_not_positive_definite():
     H = -np.eye(64)
     with pytest.raises(slim.SlimError) as e:
