@@ -262,7 +262,12 @@ def sba_search(W: np.ndarray, X: ArrayOrChunks, order: Sequence[int], group: int
     k = W.shape[1] // group
     P = sba_candidates(k)
     allocs = [allocation(order, avg_bits, p) for p in range(P)]
-    Wq = [rtn_dequant(W, a, group) for a in allocs]
+
+    def dequant(p):
+        # a candidate's quantized weights, made when used: all P of them at
+        # once would not fit in host memory for the larger layers
+        return rtn_dequant(W, allocs[p], group)
+
     kl_sum = np.zeros(P)
     ntok = 0
     for x in _as_chunks(X):
@@ -271,15 +276,18 @@ def sba_search(W: np.ndarray, X: ArrayOrChunks, order: Sequence[int], group: int
         ntok += x.shape[0]
         if not reassociate:
             for p in range(P):
-                kl_sum[p] += kl_per_token(Y, x @ Wq[p].T).sum()
+                kl_sum[p] += kl_per_token(Y, x @ dequant(p).T).sum()
         else:
-            Yq = x @ Wq[0].T
+            prev = dequant(0)
+            Yq = x @ prev.T
             kl_sum[0] += kl_per_token(Y, Yq).sum()
             for p in range(1, P):
+                cur = dequant(p)
                 for c in (order[p - 1], order[k - p]):
                     cols = slice(c * group, (c + 1) * group)
-                    Yq = Yq + x[:, cols] @ (Wq[p][:, cols] - Wq[p - 1][:, cols]).T
+                    Yq = Yq + x[:, cols] @ (cur[:, cols] - prev[:, cols]).T
                 kl_sum[p] += kl_per_token(Y, Yq).sum()
+                prev = cur
     kl = kl_sum / ntok
     p_star = int(np.argmin(kl))
     srt = np.sort(kl)
