@@ -61,6 +61,11 @@ typedef enum { SLIM_X_F32 = 0, SLIM_X_BF16 = 1 } slim_xdtype;
 const char* slim_status_string(int status);
 /* Text of the last CUDA error seen by this thread's calls ("" if none). */
 const char* slim_last_cuda_error(void);
+/* The device-side detail of this host thread's last failed call's status:
+ * for SLIM_ENOTPD the pivot index; for SLIM_ETIMEOUT the id of the bounded
+ * wait that gave up (kernel-specific); for SLIM_ERANGE where the value was
+ * found. 0 after a call that succeeded on the device. */
+int slim_last_status_detail(void);
 /* Library version string. */
 const char* slim_version(void);
 
@@ -158,6 +163,24 @@ size_t slim_sba_workspace_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int
 int slim_sba_search(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N,
                     int group, int avg_bits, const int32_t* order, double* kl, int32_t* p_star,
                     uint8_t* bits, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * slim_sba_search_split: slim_sba_search's outputs, bit for bit, from a
+ * schedule in two parts. The first part (per token tile: the outputs x W^T
+ * and the error outputs of the base allocation, over the whole input width)
+ * does not use the salience order; it runs token chunk by token chunk
+ * (chunk_tokens, a positive multiple of 256, each chunk launched on its own)
+ * and keeps each tile's state in the workspace (8 bytes per token and
+ * output). The candidate steps then continue from that state. This is the
+ * schedule slim_quantize_layer_host runs under its host-to-device copy of X
+ * (the first part of each chunk as soon as the chunk lands); here it is
+ * callable on its own. Arguments and errors as slim_sba_search; ws NULL
+ * allocates. Workspace: slim_sba_split_workspace_bytes.
+ */
+size_t slim_sba_split_workspace_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group);
+int slim_sba_search_split(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N,
+                          int group, int avg_bits, const int32_t* order, double* kl, int32_t* p_star,
+                          uint8_t* bits, int64_t chunk_tokens, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * slim_sqc: salience-weighted quantizer calibration ([P1] 组件二 SQC,

@@ -34,6 +34,13 @@ cudaError_t launch_sba_prep_w(const float* W, int64_t m, int64_t n, int64_t N, i
                               uint8_t* pw, DevStatus* st, int num_sms, int bps, cudaStream_t s);
 cudaError_t launch_sba_prep_x(const void* X, int64_t m, int64_t n, int64_t N, int xdtype, int group, int64_t t0,
                               int64_t t1, uint8_t* pw, DevStatus* st, int num_sms, int bps, cudaStream_t s);
+size_t sba_yd_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group);
+cudaError_t launch_sba_phase_a(int64_t m, int64_t n, int xdtype, int64_t N, int group, int tp0, int tp1,
+                               const uint8_t* pw, uint8_t* sw, float* yd, DevStatus* st, int num_sms,
+                               cudaStream_t s);
+cudaError_t launch_sba_steps(int64_t m, int64_t n, int xdtype, int64_t N, int group, int avg_bits,
+                             const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, const uint8_t* pw,
+                             uint8_t* sw, float* yd, DevStatus* st, int num_sms, cudaStream_t s);
 cudaError_t launch_sba_search(int64_t m, int64_t n, int xdtype, int64_t N, int group, int avg_bits,
                               const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, const uint8_t* pw,
                               uint8_t* sw, DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev);
@@ -52,6 +59,7 @@ using namespace slim;
 namespace {
 
 thread_local std::string g_last_cuda_error;
+thread_local int g_last_detail = 0;
 constexpr double kDampAlpha = 0.01;
 constexpr size_t kStatusBytes = sizeof(DevStatus);
 constexpr int kMaxGroups = 1024;
@@ -107,6 +115,7 @@ int finish(cudaStream_t s, const DevStatus* dst) {
   DevStatus hs;
   e = cudaMemcpy(&hs, dst, sizeof(hs), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e);
+  g_last_detail = hs.code ? hs.where : 0;
   if (hs.code == kStatusTimeout) return SLIM_ETIMEOUT;
   if (hs.code == kStatusNotPD) return SLIM_ENOTPD;
   if (hs.code == kStatusRangeCode) return SLIM_ERANGE;
@@ -271,6 +280,7 @@ const char* slim_status_string(int status) {
 }
 
 const char* slim_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
+int slim_last_status_detail(void) { return g_last_detail; }
 const char* slim_version(void) { return "libslim 0.1 (sm_100a)"; }
 
 int slim_num_candidates(int64_t n, int group) {
@@ -372,6 +382,44 @@ int slim_sba_search(const float* W, int64_t m, int64_t n, const void* X, int xdt
   SLIM_CUDA(cudaMemsetAsync(st, 0, kStatusBytes, s));
   SLIM_CUDA(launch_sba(W, m, n, X, xdtype, N, group, avg_bits, order, kl, p_star, bits, w.p + kStatusBytes, st,
                        sms, s, nullptr));
+  return finish(s, st);
+}
+
+size_t slim_sba_split_workspace_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
+  return kStatusBytes + al256(sba_ws_bytes(m, n, N, xdtype, group)) + al256(sba_yd_bytes(m, n, N, xdtype, group));
+}
+
+int slim_sba_search_split(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
+                          int avg_bits, const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits,
+                          int64_t chunk_tokens, void* ws, size_t ws_bytes, void* stream) {
+  if (!W || !X || !order || !bits || !aligned16(W) || !aligned16(X)) return SLIM_EINVAL;
+  if (chunk_tokens <= 0 || chunk_tokens % 256) return SLIM_EINVAL;
+  int rc = check_shape(m, n, N, xdtype, group);
+  if (rc) return rc;
+  rc = check_bits(avg_bits);
+  if (rc) return rc;
+  int sms = 0;
+  rc = device_sms(&sms);
+  if (rc) return rc;
+  if (injected("sba_search")) return SLIM_EINJECTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Workspace w;
+  rc = w.acquire(ws, ws_bytes, slim_sba_split_workspace_bytes(m, n, N, xdtype, group), s);
+  if (rc) return rc;
+  DevStatus* st = reinterpret_cast<DevStatus*>(w.p);
+  uint8_t* pw = w.p + kStatusBytes;
+  const size_t prep = sba_prep_bytes(m, n, N, xdtype, group);
+  uint8_t* sw = pw + prep;
+  float* yd = reinterpret_cast<float*>(pw + al256(sba_ws_bytes(m, n, N, xdtype, group)));
+  SLIM_CUDA(cudaMemsetAsync(st, 0, kStatusBytes, s));
+  SLIM_CUDA(launch_sba_prep_w(W, m, n, N, xdtype, group, avg_bits, pw, st, sms, 8, s));
+  for (int64_t t0 = 0; t0 < N; t0 += chunk_tokens) {
+    const int64_t t1 = (t0 + chunk_tokens < N) ? t0 + chunk_tokens : N;
+    SLIM_CUDA(launch_sba_prep_x(X, m, n, N, xdtype, group, t0, t1, pw, st, sms, 8, s));
+    SLIM_CUDA(launch_sba_phase_a(m, n, xdtype, N, group, (int)(t0 / 256), (int)((t1 + 255) / 256), pw, sw, yd, st,
+                                 sms, s));
+  }
+  SLIM_CUDA(launch_sba_steps(m, n, xdtype, N, group, avg_bits, order, kl, p_star, bits, pw, sw, yd, st, sms, s));
   return finish(s, st);
 }
 
@@ -513,6 +561,11 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
   const size_t o_z = off; off = al256(off + sb);
   const size_t o_b = off; off = al256(off + (size_t)k);
   const size_t o_ws = off; off = al256(off + L.total);
+  // bf16 X: the SBA search runs split (below), with its partials and the
+  // phase-A TMEM state in regions of their own
+  const bool split = xdtype == SLIM_X_BF16;
+  const size_t o_sw = off; off = split ? al256(off + sba_search_bytes(m, n, N, xdtype, group)) : off;
+  const size_t o_yd = off; off = split ? al256(off + sba_yd_bytes(m, n, N, xdtype, group)) : off;
   Workspace w;
   rc = w.acquire(nullptr, 0, off, s);
   if (rc) return rc;
@@ -531,8 +584,12 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
   } else {
     // bf16 X: copied in chunks of whole Hessian token slices on a copy stream;
     // each chunk's slices of H = 2 X^T X are accumulated as soon as it lands,
-    // so the tensor-core SYRK runs under the transfer. The rest of the path
-    // follows on the caller's stream.
+    // so the tensor-core SYRK runs under the transfer. So does, on the side
+    // stream, the part of the SBA search that does not depend on the salience
+    // order: each chunk's fp16 copy and its phase A (y = X W^T and the
+    // base-allocation d over the whole input width). After the inverse
+    // Hessian and the salience order, the candidate steps continue from the
+    // stored phase-A state.
     int sms = 0;
     rc = device_sms(&sms);
     if (rc) return rc;
@@ -546,6 +603,8 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
     int32_t* pstar = reinterpret_cast<int32_t*>(lw + L.off_pstar);
     uint8_t* scratch = lw + L.off_scratch;
     uint8_t* rest = lw + L.off_rest;
+    uint8_t* sw = w.p + o_sw;
+    float* yd = reinterpret_cast<float*>(w.p + o_yd);
     const int64_t stok = hessian_slice_tokens();
     const int nsl = (int)((N + stok - 1) / stok);
     const int per = (nsl + 63) / 64;               // slices per chunk: at most 64 chunks
@@ -579,6 +638,10 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
       SLIM_CUDA(launch_hessian_slices(dX, N, n, rest, st, sms, s, s0, cnt));
       SLIM_CUDA(cudaStreamWaitEvent(hc.ps, hc.ev[c], 0));
       SLIM_CUDA(launch_sba_prep_x(dX, m, n, N, xdtype, group, r0, r1, scratch, st, sms, 2, hc.ps));
+      // chunk boundaries are multiples of the slice length, so of 256 tokens:
+      // no pair of 128-token tiles straddles two chunks
+      SLIM_CUDA(launch_sba_phase_a(m, n, xdtype, N, group, (int)(r0 / 256), (int)((r1 + 255) / 256), scratch, sw,
+                                   yd, st, sms, hc.ps));
     }
     SLIM_CUDA(launch_hessian_reduce(N, n, rest, H, s));
     if (injected("hinv_diag")) return SLIM_EINJECTED;
@@ -587,8 +650,8 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
     SLIM_CUDA(launch_salience(dW, m, n, h, group, S, order, reinterpret_cast<double*>(rest), s));
     if (injected("sba_search")) return SLIM_EINJECTED;
     SLIM_CUDA(join_prepare(hc, s));
-    SLIM_CUDA(launch_sba_search(m, n, xdtype, N, group, avg_bits, order, kl, pstar, dbits, scratch, rest, st, sms, s,
-                                nullptr));
+    SLIM_CUDA(launch_sba_steps(m, n, xdtype, N, group, avg_bits, order, kl, pstar, dbits, scratch, sw, yd, st, sms,
+                               s));
     if (injected("sqc")) return SLIM_EINJECTED;
     SLIM_CUDA(launch_sqc(dW, m, n, h, dbits, group, avg_bits, lambda, n_tau, dcodes, dscale, dzero, nullptr, sms, s));
     rc = finish(s, st);

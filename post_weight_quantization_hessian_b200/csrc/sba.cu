@@ -180,6 +180,8 @@ struct SbaParams {
   int nA, nD;                    // chunks of phase A and of one delta step
   const int32_t* order;
   float* part;                   // [n_tt][n_ot][F][128], F = 2 + 2P
+  float* yd;                     // split runs: [n_tt][n_ot][e^(y-M), d][128 outputs][128 tokens]
+  int tp0;                       // first token-tile pair of this launch (n_tp pairs from there)
   DevStatus* st;
 };
 
@@ -236,8 +238,15 @@ __device__ __forceinline__ void unit_decode(const SbaParams& p, int u, int& tp, 
   const int bc = (p.n_tp - band_start < SB_BAND) ? p.n_tp - band_start : SB_BAND;
   const int r = u - band_start * p.n_ot;
   ot = r / bc;
-  tp = band_start + (r - ot * bc);
+  tp = p.tp0 + band_start + (r - ot * bc);
 }
+
+// What one launch of the scoring kernel covers.
+enum SbaMode : int {
+  kSbaAll = 0,     // phase A and every candidate step
+  kSbaPhaseA = 1,  // phase A only (it needs no order), e^(y - M) and d kept in yd
+  kSbaSteps = 2,   // candidate steps 1..P-1, starting from yd
+};
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -279,6 +288,12 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
 //               the accumulator before computing, so the next candidate's MMA
 //               overlaps the epilogue's exponentials; the two halves of a row
 //               combine their row maximum and sums through shared memory.
+// MODE splits the work in two launches (phase A does not depend on the
+// salience order, so it can run before the order exists): kSbaPhaseA also
+// stores each tile's e^(y - M) and d, exactly as they sit in TMEM after phase
+// A; kSbaSteps loads them back into TMEM and continues with step 1, so the
+// two launches together compute bit for bit what one kSbaAll launch does.
+template <int MODE>
 __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_constant__ SbaTmaps tm, SbaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -295,7 +310,10 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
   float* s_x = reinterpret_cast<float*>(s_order + ((p.k + 3) & ~3));  // [2 slots][128 rows][8]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int c = threadIdx.x; c < p.k; c += blockDim.x) s_order[c] = p.order[c];
+  constexpr int s_lo = MODE == kSbaSteps ? 1 : 0;  // the launch's steps: [s_lo, s_hi)
+  const int s_hi = MODE == kSbaPhaseA ? 1 : p.P;
+  if (MODE != kSbaPhaseA)
+    for (int c = threadIdx.x; c < p.k; c += blockDim.x) s_order[c] = p.order[c];
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int s = 0; s < 2; ++s) { mbar_init(&afull[s], 1); mbar_init(&afree[s], SB_EPI_WARPS / 2); }
@@ -321,7 +339,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
         int tp, ot;
         unit_decode(p, u, tp, ot);
         const int xrow0 = 2 * tp * SB_BM, xrow1 = xrow0 + SB_BM, brow = ot * SB_BN;
-        for (int step = 0; step < p.P && ok; ++step) {
+        for (int step = s_lo; step < s_hi && ok; ++step) {
           const ItemGeom geo = item_geom(p, s_order, step);
           const int nch = step == 0 ? p.nA : p.nD;
           for (int c = 0; c < nch; ++c) {
@@ -367,10 +385,15 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
       bool ok = true;
       const uint32_t ty0 = tbase, ty1 = tbase + 256;
       const bool dfull = p.g >= 64;  // delta chunks are whole 64-wide boxes
+      // The wait before a step's MMAs is for the epilogue's previous release of
+      // the slot; a unit's first step in kSbaSteps waits for the load of the
+      // unit's phase-A state instead, which is also the first completion of
+      // afree (in the other modes the first wait passes on the initial phase).
+      const uint32_t fpar = MODE == kSbaSteps ? 0u : 1u;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        for (int step = 0; step < p.P && ok; ++step) {
-          if (!mbar_wait(&afree[0], (cnt & 1) ^ 1, abort_flag, p.st, 220) ||
-              !mbar_wait(&afree[1], (cnt & 1) ^ 1, abort_flag, p.st, 221)) { ok = false; break; }
+        for (int step = s_lo; step < s_hi && ok; ++step) {
+          if (!mbar_wait(&afree[0], (cnt & 1) ^ fpar, abort_flag, p.st, 220) ||
+              !mbar_wait(&afree[1], (cnt & 1) ^ fpar, abort_flag, p.st, 221)) { ok = false; break; }
           tc_fence_after();
           ItemGeom geo;
           if (step > 0 && !dfull) geo = item_geom(p, s_order, step);
@@ -446,8 +469,28 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
       const int64_t col0 = (int64_t)ot * SB_BN + h * 64;
       const int nvalid = (int)((p.m - col0) > 64 ? 64 : ((p.m - col0) > 0 ? (p.m - col0) : 0));
       float* outp = p.part + ((size_t)(have ? tt : 0) * p.n_ot + ot) * F * SB_BM + r;
+      // this thread's 64 outputs of its token row in yd (e^(y - M); d at + 128 rows)
+      float* ydp = p.yd + ((size_t)(have ? tt : 0) * p.n_ot + ot) * 2 * SB_BN * SB_BM + (size_t)(h * 64) * SB_BM + r;
       float Mt = 0.f;
-      for (int step = 0; step < p.P; ++step) {
+      if (MODE == kSbaSteps) {
+        // phase A's TMEM contents back in place; the arrival on afree hands the
+        // slot to the first candidate step's MMAs (a unit's last step does not
+        // release the slot in this mode: this load does)
+        uint32_t v[64];
+#pragma unroll
+        for (int j = 0; j < 64; ++j) v[j] = have ? __float_as_uint(ydp[(size_t)j * SB_BM]) : 0u;
+        tmem_st32(ty, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_st32(ty + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+#pragma unroll
+        for (int j = 0; j < 64; ++j) v[j] = have ? __float_as_uint(ydp[(size_t)(SB_BN + j) * SB_BM]) : 0u;
+        tmem_st32(td, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_st32(td + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afree[slot]);
+      }
+      for (int step = s_lo; step < s_hi; ++step) {
         if (!mbar_wait(&afull[slot], cnt & 1, abort_flag, p.st, 240 + slot)) { ok = false; break; }
         tc_fence_after();
         uint32_t v[64];
@@ -475,6 +518,10 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           }
           tmem_st32(ty, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
           tmem_st32(ty + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          if (MODE == kSbaPhaseA && have) {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) ydp[(size_t)j * SB_BM] = __uint_as_float(v[j]);
+          }
           tc_wait_st();
           Mt = mx;
         }
@@ -483,7 +530,11 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
         tmem_ld32(td, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
         tmem_ld32(td + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tc_wait_ld();
-        const bool last = step == p.P - 1;
+        if (MODE == kSbaPhaseA && have) {
+#pragma unroll
+          for (int j = 0; j < 64; ++j) ydp[(size_t)(SB_BN + j) * SB_BM] = __uint_as_float(v[j]);
+        }
+        const bool last = step == s_hi - 1;
         if (!last) {
           tc_fence_before();
           __syncwarp();
@@ -509,7 +560,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
         float sq0, sq1, a0, a1;
         f2_unpack(sqp, sq0, sq1);
         f2_unpack(ap, a0, a1);
-        if (last) {
+        if (last && MODE != kSbaSteps) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&afree[slot]);
@@ -704,49 +755,96 @@ cudaError_t launch_sba_prep_x(const void* X, int64_t m, int64_t n, int64_t N, in
   return cudaGetLastError();
 }
 
+size_t sba_yd_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
+  const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
+  return (size_t)pl.n_tt * pl.n_ot * 2 * SB_BN * SB_BM * sizeof(float);
+}
+
+// One scoring launch over token-tile pairs [tp0, tp1) on the prepared operands
+// (pw) and the search region (sw).
+template <int MODE>
+static cudaError_t launch_score(const SbaPlan& pl, int64_t m, int64_t n, int64_t N, int group, const int32_t* order,
+                                const uint8_t* pw, uint8_t* sw, float* yd, int tp0, int tp1, DevStatus* st,
+                                int num_sms, cudaStream_t s, cudaEvent_t* kev) {
+  if (pl.k > SB_MAX_K || tp0 < 0 || tp1 > pl.n_tp || tp1 < tp0) return cudaErrorInvalidValue;
+  if (tp1 == tp0) return cudaSuccess;
+  SbaTmaps tm;
+  bool ok = make_tmap_f16(&tm.x, pw + pl.off_xc, (uint64_t)(n * pl.ksplit), (uint64_t)N, SB_BK, SB_BM);
+  ok = ok && make_tmap_f16(&tm.wb, pw + pl.off_wb, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
+  ok = ok && make_tmap_f16(&tm.e0, pw + pl.off_e0, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
+  ok = ok && make_tmap_f16(&tm.dp, pw + pl.off_dp, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
+  ok = ok && make_tmap_f16(&tm.dm, pw + pl.off_dm, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
+  if (!ok) return cudaErrorInvalidValue;
+  SbaParams p;
+  p.N = N; p.m = m; p.n = n; p.g = group; p.k = pl.k; p.P = pl.P; p.ksplit = pl.ksplit;
+  p.n_tt = pl.n_tt; p.n_tp = tp1 - tp0; p.n_ot = pl.n_ot; p.stages = pl.stages; p.nA = pl.nA; p.nD = pl.nD;
+  p.order = order; p.part = reinterpret_cast<float*>(sw); p.yd = yd; p.tp0 = tp0; p.st = st;
+  static bool attr = false;
+  if (!attr) {  // the plan's shared memory never exceeds this bound
+    cudaError_t e = cudaFuncSetAttribute(sba_score_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         227 * 1024);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int units = p.n_tp * pl.n_ot;
+  const int grid = units < num_sms ? units : num_sms;
+  if (kev) cudaEventRecord(kev[0], s);
+  sba_score_kernel<MODE><<<grid, SB_THREADS, pl.smem, s>>>(tm, p);
+  if (kev) cudaEventRecord(kev[1], s);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// Per-token KL from the partials, its means over tokens, p* and the bits.
+static cudaError_t launch_merge_final(const SbaPlan& pl, int64_t N, int avg_bits, const int32_t* order, double* kl,
+                                      int32_t* p_star, uint8_t* bits, uint8_t* sw, cudaStream_t s) {
+  float* part = reinterpret_cast<float*>(sw);
+  double* klp = reinterpret_cast<double*>(sw + (pl.off_klp - pl.off_part));
+  const size_t msmem = (size_t)pl.n_ot * SB_BM * sizeof(float);
+  if (msmem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(sba_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+    if (e != cudaSuccess) return e;
+  }
+  sba_merge_kernel<<<pl.n_tt, SB_BM, msmem, s>>>(part, pl.n_ot, pl.P, N, pl.n_tt, klp);
+  sba_final_kernel<<<1, 256, 0, s>>>(klp, pl.n_tt, pl.P, N, order, pl.k, avg_bits, kl, p_star, bits);
+  count_launches(2);
+  return cudaGetLastError();
+}
+
 // Scoring, merge and final selection on the prepared operands (pw) with the
 // search region (sw: sba_search_bytes) for the partial sums.
 cudaError_t launch_sba_search(int64_t m, int64_t n, int xdtype, int64_t N, int group, int avg_bits,
                               const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, const uint8_t* pw,
                               uint8_t* sw, DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev) {
   const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
-  if (pl.k > SB_MAX_K) return cudaErrorInvalidValue;
-  const __half* Wb = reinterpret_cast<const __half*>(pw + pl.off_wb);
-  const __half* E0 = reinterpret_cast<const __half*>(pw + pl.off_e0);
-  const __half* Dp = reinterpret_cast<const __half*>(pw + pl.off_dp);
-  const __half* Dm = reinterpret_cast<const __half*>(pw + pl.off_dm);
-  const __half* Xc = reinterpret_cast<const __half*>(pw + pl.off_xc);
-  float* part = reinterpret_cast<float*>(sw);
-  double* klp = reinterpret_cast<double*>(sw + (pl.off_klp - pl.off_part));
-  const void* xptr = Xc;
-  SbaTmaps tm;
-  bool ok = make_tmap_f16(&tm.x, xptr, (uint64_t)(n * pl.ksplit), (uint64_t)N, SB_BK, SB_BM);
-  ok = ok && make_tmap_f16(&tm.wb, Wb, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
-  ok = ok && make_tmap_f16(&tm.e0, E0, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
-  ok = ok && make_tmap_f16(&tm.dp, Dp, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
-  ok = ok && make_tmap_f16(&tm.dm, Dm, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
-  if (!ok) return cudaErrorInvalidValue;
-
-  SbaParams p;
-  p.N = N; p.m = m; p.n = n; p.g = group; p.k = pl.k; p.P = pl.P; p.ksplit = pl.ksplit;
-  p.n_tt = pl.n_tt; p.n_tp = pl.n_tp; p.n_ot = pl.n_ot; p.stages = pl.stages; p.nA = pl.nA; p.nD = pl.nD;
-  p.order = order; p.part = part; p.st = st;
-  cudaError_t e = cudaFuncSetAttribute(sba_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
+  cudaError_t e = launch_score<kSbaAll>(pl, m, n, N, group, order, pw, sw, nullptr, 0, pl.n_tp, st, num_sms, s, kev);
   if (e != cudaSuccess) return e;
-  const int units = pl.n_tp * pl.n_ot;
-  const int grid = units < num_sms ? units : num_sms;
-  if (kev) cudaEventRecord(kev[0], s);
-  sba_score_kernel<<<grid, SB_THREADS, pl.smem, s>>>(tm, p);
-  if (kev) cudaEventRecord(kev[1], s);
-  const size_t msmem = (size_t)pl.n_ot * SB_BM * sizeof(float);
-  if (msmem > 48 * 1024) {
-    e = cudaFuncSetAttribute(sba_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+  return launch_merge_final(pl, N, avg_bits, order, kl, p_star, bits, sw, s);
+}
+
+// Split search, first part: phase A for token-tile pairs [tp0, tp1) (pairs of
+// 128-token tiles); it needs only the prepared operands of those tokens.
+// Writes the pairs' phase-A partials into sw and their TMEM state into yd
+// (sba_yd_bytes).
+cudaError_t launch_sba_phase_a(int64_t m, int64_t n, int xdtype, int64_t N, int group, int tp0, int tp1,
+                               const uint8_t* pw, uint8_t* sw, float* yd, DevStatus* st, int num_sms,
+                               cudaStream_t s) {
+  const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
+  return launch_score<kSbaPhaseA>(pl, m, n, N, group, nullptr, pw, sw, yd, tp0, tp1, st, num_sms, s, nullptr);
+}
+
+// Split search, second part, once every pair's phase A is in sw and yd: the
+// candidate steps, merge and final selection.
+cudaError_t launch_sba_steps(int64_t m, int64_t n, int xdtype, int64_t N, int group, int avg_bits,
+                             const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, const uint8_t* pw,
+                             uint8_t* sw, float* yd, DevStatus* st, int num_sms, cudaStream_t s) {
+  const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
+  if (pl.P > 1) {
+    cudaError_t e = launch_score<kSbaSteps>(pl, m, n, N, group, order, pw, sw, yd, 0, pl.n_tp, st, num_sms, s,
+                                            nullptr);
     if (e != cudaSuccess) return e;
   }
-  sba_merge_kernel<<<pl.n_tt, SB_BM, msmem, s>>>(part, pl.n_ot, pl.P, N, pl.n_tt, klp);
-  sba_final_kernel<<<1, 256, 0, s>>>(klp, pl.n_tt, pl.P, N, order, pl.k, avg_bits, kl, p_star, bits);
-  count_launches(3);
-  return cudaGetLastError();
+  return launch_merge_final(pl, N, avg_bits, order, kl, p_star, bits, sw, s);
 }
 
 cudaError_t launch_sba(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,

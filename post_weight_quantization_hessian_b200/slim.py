@@ -28,6 +28,9 @@ STATUS = {0: "SLIM_OK", 1: "SLIM_EINVAL", 2: "SLIM_ENOMEM", 3: "SLIM_ECUDA", 4: 
 class SlimError(RuntimeError):
     def __init__(self, status: int, where: str, detail: str = ""):
         self.status = status
+        self.device_detail = _lib().slim_last_status_detail()
+        if self.device_detail:
+            detail = (detail + " " if detail else "") + f"[device detail {self.device_detail}]"
         super().__init__(f"{where}: {STATUS.get(status, status)} ({_lib().slim_status_string(status).decode()})"
                          + (f" {detail}" if detail else ""))
 
@@ -44,6 +47,7 @@ class SlimDiag(ctypes.Structure):
 _SIGS = {
     "slim_status_string": (ctypes.c_char_p, [i32]),
     "slim_last_cuda_error": (ctypes.c_char_p, []),
+    "slim_last_status_detail": (i32, []),
     "slim_version": (ctypes.c_char_p, []),
     "slim_num_candidates": (i32, [i64, i32]),
     "slim_row_words": (i64, [i64, i32]),
@@ -57,6 +61,8 @@ _SIGS = {
     "slim_salience_noalloc": (i32, [vp, i64, i64, vp, i32, vp, vp, vp]),
     "slim_sba_workspace_bytes": (sz, [i64, i64, i64, i32, i32]),
     "slim_sba_search": (i32, [vp, i64, i64, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp]),
+    "slim_sba_split_workspace_bytes": (sz, [i64, i64, i64, i32, i32]),
+    "slim_sba_search_split": (i32, [vp, i64, i64, vp, i32, i64, i32, i32, vp, vp, vp, vp, i64, vp, sz, vp]),
     "slim_sqc": (i32, [vp, i64, i64, vp, vp, i32, i32, dbl, i32, vp, vp, vp, vp, vp]),
     "slim_workspace_bytes": (sz, [i64, i64, i64, i32, i32, i32]),
     "slim_quantize_layer": (i32, [vp, i64, i64, vp, i32, i64, i32, i32, dbl, i32, vp, vp, vp, vp, vp, sz, vp]),
@@ -209,6 +215,22 @@ def slim_sba_search(W: torch.Tensor, X: torch.Tensor, group: int, avg_bits: int,
     wsb = ws.numel() * ws.element_size() if isinstance(ws, torch.Tensor) else 0
     _check(_lib().slim_sba_search(_ptr(W), m, n, _ptr(X), _xdtype(X), N, group, avg_bits, _ptr(order), _ptr(kl),
                                   _ptr(p_star), _ptr(bits), _ptr(ws), wsb, _stream(stream)), "slim_sba_search")
+    return kl, p_star, bits
+
+
+def slim_sba_search_split(W: torch.Tensor, X: torch.Tensor, group: int, avg_bits: int, order: torch.Tensor,
+                          chunk_tokens: int, ws=None, stream=None):
+    m, n = W.shape
+    N = X.shape[0]
+    k = n // group
+    P = k // 2 + 1
+    kl = torch.empty(P, dtype=torch.float64, device=W.device)
+    p_star = torch.empty(1, dtype=torch.int32, device=W.device)
+    bits = torch.empty(k, dtype=torch.uint8, device=W.device)
+    wsb = ws.numel() * ws.element_size() if isinstance(ws, torch.Tensor) else 0
+    _check(_lib().slim_sba_search_split(_ptr(W), m, n, _ptr(X), _xdtype(X), N, group, avg_bits, _ptr(order),
+                                        _ptr(kl), _ptr(p_star), _ptr(bits), int(chunk_tokens), _ptr(ws), wsb,
+                                        _stream(stream)), "slim_sba_search_split")
     return kl, p_star, bits
 
 

@@ -147,6 +147,36 @@ def test_sba_search(kw):
     assert b.sum() == s.k * s.avg_bits
 
 
+SPLIT_CASES = [(kw, 256) for kw in SBA_CASES] + [
+    (dict(m=384, n=512, N=5000, group=64), 512),     # 40 token tiles: chunks of 2 pairs, ragged last tile
+    (dict(m=128, n=128, N=600, group=128), 256),     # k = 1: phase A only, no candidate step
+    (dict(m=130, n=256, N=3000, group=32, avg_bits=3), 1024),
+]
+
+
+@pytest.mark.parametrize("kw, chunk", SPLIT_CASES)
+def test_sba_search_split_matches_one_pass(kw, chunk):
+    """Phase A per token chunk, its TMEM state stored, the candidate steps resumed
+    from it: the same KL, p* and bits as the one-pass search, bit for bit."""
+    s = spec(**kw)
+    W, Xh, Wd, Xd = device_inputs(s)
+    order = torch.from_numpy(np.random.default_rng(s.seed).permutation(s.k).astype(np.int32)).cuda()
+    kl1, p1, b1 = slim.slim_sba_search(Wd, Xd, s.group, s.avg_bits, order)
+    kl2, p2, b2 = slim.slim_sba_search_split(Wd, Xd, s.group, s.avg_bits, order, chunk)
+    assert np.array_equal(kl1.cpu().numpy().view(np.uint64), kl2.cpu().numpy().view(np.uint64))
+    assert int(p1.item()) == int(p2.item())
+    assert np.array_equal(b1.cpu().numpy(), b2.cpu().numpy())
+
+
+def test_sba_search_split_rejects_unaligned_chunks():
+    s = spec()
+    W, Xh, Wd, Xd = device_inputs(s)
+    order = torch.arange(s.k, dtype=torch.int32, device="cuda")
+    with pytest.raises(slim.SlimError) as e:
+        slim.slim_sba_search_split(Wd, Xd, s.group, s.avg_bits, order, 384)
+    assert e.value.status == 1
+
+
 def test_sqc_larger_layer():
     """1M weights x 50 candidates: every quotient of the calibration loop exercised."""
     s = spec(m=1024, n=1024, group=64, avg_bits=3, seed=21)
