@@ -398,11 +398,14 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           ItemGeom geo;
           if (step > 0 && !dfull) geo = item_geom(p, s_order, step);
           const int nch = step == 0 ? p.nA : p.nD;
-          // A shared-memory access by this thread waits for its MMAs to drain
-          // (about 190 cycles), so each wait is made to cover as much work as
-          // possible: right after the blocking wait on a chunk's stage, the next
-          // chunk of the same step is tested (cheap, nothing in flight) and, if
-          // its stage is full too, both chunks go out behind the one wait.
+          // A shared-memory access by this thread while its MMAs are in flight
+          // waits for them to drain (about 380 cycles: the queue holds only a few
+          // MMAs), so each wait is made to cover two chunks where it can: right
+          // after the blocking wait on a chunk's stage, the next chunk of the
+          // same step is tested (cheap, nothing new in flight) and, if its stage
+          // is full too, both chunks go out behind the one wait. (Taking all
+          // three stages at once is slower: no stage is then being refilled
+          // while the MMAs run.)
           for (int c = 0; c < nch;) {
             if (!mbar_wait(&full[st], ph, abort_flag, p.st, 230 + st)) { ok = false; break; }
             int st2 = st + 1;
@@ -542,20 +545,35 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
         }
         uint64_t sqp = 0, ap = 0;  // packed (even, odd column) sums
         const uint64_t kc2 = f2_pack(kC1, kC1);
+        // e^(y - M) in 8-column pieces. In the split launches the pieces are
+        // double-buffered (the load of the next one is in flight while this one
+        // is consumed); the one-pass launch, whose step-0 code already holds
+        // more registers, loads them one at a time. Same arithmetic either way.
+        constexpr int NB = MODE == kSbaAll ? 1 : 2;
+        uint32_t ev[NB][8];
+        if (NB == 2) {
+          tmem_ld8(ty, ev[0]);
+          tc_wait_ld8(ev[0]);
+        }
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
-          uint32_t ev[8];
-          tmem_ld8(ty + cc * 8, ev);
-          tc_wait_ld();
+          uint32_t (&cur)[8] = ev[cc % NB];
+          if (NB == 1) {
+            tmem_ld8(ty + cc * 8, cur);
+            tc_wait_ld8(cur);
+          } else if (cc + 1 < 8) {
+            tmem_ld8(ty + (cc + 1) * 8, ev[(cc + 1) % NB]);
+          }
 #pragma unroll
           for (int j = 0; j < 8; j += 2) {
-            const uint64_t ey = f2_pack(__uint_as_float(ev[j]), __uint_as_float(ev[j + 1]));
+            const uint64_t ey = f2_pack(__uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
             const uint64_t dd = f2_pack(__uint_as_float(v[cc * 8 + j]), __uint_as_float(v[cc * 8 + j + 1]));
             float x0, x1;
             f2_unpack(f2_mul(dd, kc2), x0, x1);
             sqp = f2_fma(ey, f2_pack(ex2(x0), ex2(x1)), sqp);
             ap = f2_fma(ey, dd, ap);
           }
+          if (NB == 2 && cc + 1 < 8) tc_wait_ld8(ev[(cc + 1) % NB]);
         }
         float sq0, sq1, a0, a1;
         f2_unpack(sqp, sq0, sq1);
