@@ -245,13 +245,14 @@ struct JoinOnExit {
 
 // Forks onto the side stream, once everything queued on s so far is done,
 // the preparation of the SBA weight operands and (X non-null) of all of X,
-// at bps blocks per SM. Join with join_prepare.
+// at bps_w and bps_x blocks per SM. Join with join_prepare.
 cudaError_t fork_prepare(HostCopy& side, const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N,
-                         int group, int avg_bits, uint8_t* pw, DevStatus* st, int sms, int bps, cudaStream_t s) {
+                         int group, int avg_bits, uint8_t* pw, DevStatus* st, int sms, int bps_w, int bps_x,
+                         cudaStream_t s) {
   cudaError_t e = cudaEventRecord(side.pe[0], s);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(side.ps, side.pe[0], 0);
-  if (e == cudaSuccess) e = launch_sba_prep_w(W, m, n, N, xdtype, group, avg_bits, pw, st, sms, bps, side.ps);
-  if (e == cudaSuccess && X) e = launch_sba_prep_x(X, m, n, N, xdtype, group, 0, N, pw, st, sms, bps, side.ps);
+  if (e == cudaSuccess) e = launch_sba_prep_w(W, m, n, N, xdtype, group, avg_bits, pw, st, sms, bps_w, side.ps);
+  if (e == cudaSuccess && X) e = launch_sba_prep_x(X, m, n, N, xdtype, group, 0, N, pw, st, sms, bps_x, side.ps);
   return e;
 }
 cudaError_t join_prepare(HostCopy& side, cudaStream_t s) {
@@ -495,9 +496,10 @@ int slim_quantize_layer_ex(const float* W, int64_t m, int64_t n, const void* X, 
     if (injected("hessian")) return SLIM_EINJECTED;
     SLIM_CUDA(launch_hessian(X, xdtype, N, n, H, rest, st, sms, s, kev_h));
     rec(1);
-    // beside the latency-bound inverse: one block per SM leaves each SM the
-    // registers and shared memory of one factorization CTA plus the updates
-    SLIM_CUDA(fork_prepare(side, W, m, n, X, xdtype, N, group, avg_bits, scratch, st, sms, 1, s));
+    // beside the latency-bound inverse, at most 16K registers per SM (one
+    // weight-operand block or two conversion blocks), so that a factorization
+    // CTA (about 47K) still fits on every SM
+    SLIM_CUDA(fork_prepare(side, W, m, n, X, xdtype, N, group, avg_bits, scratch, st, sms, 1, 2, s));
     if (injected("hinv_diag")) return SLIM_EINJECTED;
     SLIM_CUDA(launch_hinv(H, n, kDampAlpha, h, reinterpret_cast<double*>(rest), st, s));
     rec(2);
@@ -628,7 +630,7 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
     }
     // W (copied on s above) is resident: its operands are prepared on the
     // side stream, then each chunk of X is converted there as it lands
-    SLIM_CUDA(fork_prepare(hc, dW, m, n, nullptr, xdtype, N, group, avg_bits, scratch, st, sms, 2, s));
+    SLIM_CUDA(fork_prepare(hc, dW, m, n, nullptr, xdtype, N, group, avg_bits, scratch, st, sms, 2, 2, s));
     if (injected("hessian")) return SLIM_EINJECTED;
     for (int c = 0; c < nch; ++c) {
       const int64_t r0 = (int64_t)c * per * stok;

@@ -61,54 +61,68 @@ __device__ __forceinline__ __half to_half_checked(float v, DevStatus* st, int wh
   return __float2half_rn(v);
 }
 
+// Weight-side operands. W is read as float4: a lane holds 4 consecutive
+// weights, a group of G spans G/4 adjacent lanes (G divides 128 and n, so a
+// group never leaves its lanes or its row), and each output array gets one
+// 8-byte store per lane. Per group: fp32 min/max, then per level b-1, b, b+1
+// the fp64 min-max RTN value.
 template <int G>
-__global__ void __launch_bounds__(256) sba_prep_kernel(const float* __restrict__ W, int64_t m, int64_t n,
-                                                       int avg_bits, __half* __restrict__ Wb, __half* __restrict__ E0,
-                                                       __half* __restrict__ Dp, __half* __restrict__ Dm,
+__global__ void __launch_bounds__(256) sba_prep_kernel(const float4* __restrict__ W, int64_t total4, int avg_bits,
+                                                       uint2* __restrict__ Wb, uint2* __restrict__ E0,
+                                                       uint2* __restrict__ Dp, uint2* __restrict__ Dm,
                                                        DevStatus* st) {
-  constexpr int E = G / 32;
+  constexpr int LPG = G / 4;  // lanes per group
   const int lane = threadIdx.x & 31;
-  const int64_t k = n / G;
-  const int64_t pairs = m * k;
-  const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t pr = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); pr < pairs; pr += wstride) {
-    const int64_t i = pr / k, c = pr - (pr / k) * k;
-    const int64_t base = i * n + c * G;
-    float w[E];
-    float lo = 0.f, hi = 0.f;
+  const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5) * 32;
+  for (int64_t base = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 32; base < total4;
+       base += wstride) {
+    const int64_t e = base + lane;
+    const bool on = e < total4;  // whole groups are on or off together (the total is a multiple of G)
+    const float4 v4 = on ? W[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float w[4] = {v4.x, v4.y, v4.z, v4.w};
+    float lo = fminf(fminf(w[0], w[1]), fminf(w[2], w[3]));
+    float hi = fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3]));
 #pragma unroll
-    for (int r = 0; r < E; ++r) {
-      w[r] = W[base + lane + 32 * r];
-      lo = r ? fminf(lo, w[r]) : w[r];
-      hi = r ? fmaxf(hi, w[r]) : w[r];
+    for (int o = LPG / 2; o > 0; o >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
     }
-    lo = warp_min(lo);
-    hi = warp_max(hi);
+    if (!on) continue;
     const double dlo = lo, dhi = hi;
     const bool deg = (dhi == dlo);
-    double wh[3][E];
+    double wh[3][4];
 #pragma unroll
     for (int l = 0; l < 3; ++l) {
       const int b = avg_bits - 1 + l;
       const double qmax = (double)((1 << b) - 1);
       const double s0 = deg ? 1.0 : (dhi - dlo) / qmax;
       const double z0 = deg ? -dlo : -dlo / s0;
+      // w / s0 correctly rounded from one IEEE reciprocal and Markstein's final
+      // division step (P. Markstein, IBM J. Res. Dev. 34(1), 1990): exact while
+      // nothing overflows or underflows, which fp32 weights and scales ensure
+      const double y = 1.0 / s0;
 #pragma unroll
-      for (int r = 0; r < E; ++r) {
-        double q = rint((double)w[r] / s0 + z0);
+      for (int r = 0; r < 4; ++r) {
+        const double wd = w[r];
+        const double q0 = wd * y;
+        double q = rint(fma(fma(-q0, s0, wd), y, q0) + z0);
         q = fmin(fmax(q, 0.0), qmax);
-        wh[l][r] = deg ? (double)w[r] : s0 * (q - z0);
+        wh[l][r] = deg ? wd : s0 * (q - z0);
       }
     }
+    __half o0[4], o1[4], o2[4], o3[4];
 #pragma unroll
-    for (int r = 0; r < E; ++r) {
-      const int64_t o = base + lane + 32 * r;
+    for (int r = 0; r < 4; ++r) {
       const double wd = w[r];
-      Wb[o] = to_half_checked(w[r] * kOpScale, st, 300);
-      E0[o] = to_half_checked((float)(wh[1][r] - wd) * kOpScale, st, 301);
-      Dp[o] = to_half_checked((float)(wh[2][r] - wh[1][r]) * kOpScale, st, 302);
-      Dm[o] = to_half_checked((float)(wh[0][r] - wh[1][r]) * kOpScale, st, 303);
+      o0[r] = to_half_checked(w[r] * kOpScale, st, 300);
+      o1[r] = to_half_checked((float)(wh[1][r] - wd) * kOpScale, st, 301);
+      o2[r] = to_half_checked((float)(wh[2][r] - wh[1][r]) * kOpScale, st, 302);
+      o3[r] = to_half_checked((float)(wh[0][r] - wh[1][r]) * kOpScale, st, 303);
     }
+    Wb[e] = *reinterpret_cast<const uint2*>(o0);
+    E0[e] = *reinterpret_cast<const uint2*>(o1);
+    Dp[e] = *reinterpret_cast<const uint2*>(o2);
+    Dm[e] = *reinterpret_cast<const uint2*>(o3);
   }
 }
 
@@ -741,13 +755,16 @@ cudaError_t launch_sba_prep_w(const float* W, int64_t m, int64_t n, int64_t N, i
   __half* E0 = reinterpret_cast<__half*>(pw + pl.off_e0);
   __half* Dp = reinterpret_cast<__half*>(pw + pl.off_dp);
   __half* Dm = reinterpret_cast<__half*>(pw + pl.off_dm);
-  const int64_t pairs = m * pl.k;
-  int pgrid = (int)((pairs + 7) / 8);
-  if (pgrid > num_sms * 2 * bps) pgrid = num_sms * 2 * bps;
+  const int64_t total4 = m * n / 4;              // n is a multiple of 32
+  int pgrid = (int)((total4 + 255) / 256);        // 8 warps x 32 float4 per block and pass
+  if (pgrid > num_sms * bps) pgrid = num_sms * bps;
+  const float4* W4 = reinterpret_cast<const float4*>(W);
+  uint2 *b0 = reinterpret_cast<uint2*>(Wb), *b1 = reinterpret_cast<uint2*>(E0), *b2 = reinterpret_cast<uint2*>(Dp),
+        *b3 = reinterpret_cast<uint2*>(Dm);
   switch (group) {
-    case 32: sba_prep_kernel<32><<<pgrid, 256, 0, s>>>(W, m, n, avg_bits, Wb, E0, Dp, Dm, st); break;
-    case 64: sba_prep_kernel<64><<<pgrid, 256, 0, s>>>(W, m, n, avg_bits, Wb, E0, Dp, Dm, st); break;
-    case 128: sba_prep_kernel<128><<<pgrid, 256, 0, s>>>(W, m, n, avg_bits, Wb, E0, Dp, Dm, st); break;
+    case 32: sba_prep_kernel<32><<<pgrid, 256, 0, s>>>(W4, total4, avg_bits, b0, b1, b2, b3, st); break;
+    case 64: sba_prep_kernel<64><<<pgrid, 256, 0, s>>>(W4, total4, avg_bits, b0, b1, b2, b3, st); break;
+    case 128: sba_prep_kernel<128><<<pgrid, 256, 0, s>>>(W4, total4, avg_bits, b0, b1, b2, b3, st); break;
     default: return cudaErrorInvalidValue;
   }
   count_launches(1);
