@@ -9,8 +9,10 @@
 //
 // One warp owns one (row, group). Phase 1 (lanes over elements): load the
 // group, moments, 3-sigma mask, min/max, element salience; stage w and delta
-// in shared memory. Phase 2 (lanes over tau): lane l scores tau_l, tau_{l+32},
-// ... over all g elements. Every score is fp64 with the operation order of the
+// in shared memory, the masked elements first (a stable partition, so each
+// class is summed in column order without a per-element test). Phase 2
+// (lanes over tau): lane l scores tau_l, tau_{l+32}, ... over all g elements;
+// the code clamp runs on a 32-bit integer (round half to even, as rint). Every score is fp64 with the operation order of the
 // definition (IEEE division and rint), so the chosen tau matches a float64
 // evaluation except where two candidates' errors tie to rounding. Phase 3
 // (lanes over elements): codes at the chosen tau, bytes to shared memory, then
@@ -41,7 +43,6 @@ sqc_kernel(const float* __restrict__ W, int64_t m, int64_t n, const double* __re
   constexpr int E = G / 32;  // elements per lane
   __shared__ double s_w[kSqcWarps][G];
   __shared__ double s_d[kSqcWarps][G];
-  __shared__ uint8_t s_msk[kSqcWarps][G];
   __shared__ uint8_t s_q[kSqcWarps][G];
 
   const int lane = threadIdx.x & 31;
@@ -55,6 +56,7 @@ sqc_kernel(const float* __restrict__ W, int64_t m, int64_t n, const double* __re
     const int c = (int)(pr - i * k);
     const int b = bits[c];
     const double qmax = (double)((1 << b) - 1);
+    const int qmaxi = (1 << b) - 1;
     const float* wp = W + i * n + (int64_t)c * G;
 
     // ---- phase 1: moments, mask, range, salience
@@ -81,20 +83,32 @@ sqc_kernel(const float* __restrict__ W, int64_t m, int64_t n, const double* __re
     var = warp_sum(var) / (double)G;
     const double sd = sqrt(var);
     const double tlo = mu - 3.0 * sd, thi = mu + 3.0 * sd;
+    // stable partition in shared memory: the masked (salient) elements first,
+    // each class in column order, so the tau loop sums each class without a
+    // per-element test, in the same order as before
+    bool mk[E];
     int ns = 0;
 #pragma unroll
     for (int r = 0; r < E; ++r) {
-      const int j = lane + 32 * r;
-      const double hj = h[(int64_t)c * G + j];
-      const bool mk = (w[r] < tlo) || (w[r] > thi);
-      ns += mk ? 1 : 0;
-      s_w[wib][j] = w[r];
-      s_d[wib][j] = (w[r] * w[r]) / (hj * hj);
-      s_msk[wib][j] = mk ? 1 : 0;
+      mk[r] = (w[r] < tlo) || (w[r] > thi);
+      ns += __popc(__ballot_sync(0xffffffffu, mk[r]));
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ns += __shfl_xor_sync(0xffffffffu, ns, o);
     const int nu = G - ns;
+    {
+      const uint32_t lt = (1u << lane) - 1u;
+      int before_m = 0;
+#pragma unroll
+      for (int r = 0; r < E; ++r) {
+        const int j = lane + 32 * r;
+        const uint32_t bm = __ballot_sync(0xffffffffu, mk[r]);
+        const int pm = before_m + __popc(bm & lt);              // masked elements before j
+        const int pos = mk[r] ? pm : ns + (j - pm);             // unmasked: after all masked
+        const double hj = h[(int64_t)c * G + j];
+        s_w[wib][pos] = w[r];
+        s_d[wib][pos] = (w[r] * w[r]) / (hj * hj);
+        before_m += __popc(bm);
+      }
+    }
     __syncwarp();
 
     const bool deg = (hi == lo);
@@ -112,18 +126,19 @@ sqc_kernel(const float* __restrict__ W, int64_t m, int64_t n, const double* __re
         const double s = tau * s0;
         const double y = 1.0 / s;
         double es = 0.0, eu = 0.0;
-#pragma unroll 4
-        for (int j = 0; j < G; ++j) {
+        auto term = [&](int j) {
           const double wj = s_w[wib][j];
           const double q0 = wj * y;
           const double quot = fma(fma(-q0, s, wj), y, q0);   // = RN(wj / s)
-          double q = rint(quot + z0);
-          q = (q < 0.0) ? 0.0 : q;   // clamp by selects: the fp64 min/max are slower here
-          q = (q > qmax) ? qmax : q;
+          int qi = __double2int_rn(quot + z0);   // round half to even, as rint
+          qi = qi < 0 ? 0 : (qi > qmaxi ? qmaxi : qi);
+          const double q = (double)qi;
           const double e = wj - s * (q - z0);
-          const double v = s_d[wib][j] * (e * e);
-          if (s_msk[wib][j]) es += v; else eu += v;
-        }
+          return s_d[wib][j] * (e * e);
+        };
+        for (int j = 0; j < ns; ++j) es += term(j);
+#pragma unroll 4
+        for (int j = ns; j < G; ++j) eu += term(j);
         double err = (nu > 0 ? eu / (double)nu : 0.0);
         if (ns > 0) err = err + es / (double)ns;
         if (err < best_e) { best_e = err; best_t = t; }
