@@ -8,6 +8,7 @@
 // - thin inline-PTX wrappers for mbarrier, TMA tiled loads (no multicast) and
 //   the tcgen05 tensor-core / tensor-memory instructions.
 #pragma once
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -16,6 +17,16 @@
 #endif
 
 namespace slim {
+
+// Kernel attributes set with cudaFuncSetAttribute belong to the current
+// device, so "already set" is remembered per device (bit dev of a mask).
+inline bool attr_pending(std::atomic<uint64_t>& mask, uint64_t& bit) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  bit = 1ull << (dev & 63);
+  return (mask.load(std::memory_order_acquire) & bit) == 0;
+}
+
 
 // Host: running count of kernels this library has launched (all threads).
 void count_launches(int k);

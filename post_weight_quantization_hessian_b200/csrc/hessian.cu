@@ -295,11 +295,12 @@ cudaError_t launch_hessian_slices(const void* X, int64_t N, int64_t n, void* par
   const SyrkPlan pl = syrk_plan_bf16(N, n);
   CUtensorMap tm;
   if (!make_tmap_bf16(&tm, X, (uint64_t)n, (uint64_t)N, 64, 64)) return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
+  static std::atomic<uint64_t> attr{0};
+  uint64_t bit = 0;
+  if (attr_pending(attr, bit)) {
     cudaError_t e = cudaFuncSetAttribute(syrk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM);
     if (e != cudaSuccess) return e;
-    attr = true;
+    attr.fetch_or(bit);
   }
   SyrkParams p;
   p.N = N; p.n = n; p.nblk = pl.nblk; p.npairs = pl.npairs; p.nslices = pl.nslices;
@@ -329,11 +330,12 @@ cudaError_t launch_hessian(const void* X, int xdtype, int64_t N, int64_t n, doub
     const SyrkPlan pl = syrk_plan_bf16(N, n);
     CUtensorMap tm;
     if (!make_tmap_bf16(&tm, X, (uint64_t)n, (uint64_t)N, 64, 64)) return cudaErrorInvalidValue;
-    static bool attr = false;
-    if (!attr) {
+    static std::atomic<uint64_t> attr{0};
+    uint64_t bit = 0;
+    if (attr_pending(attr, bit)) {
       cudaError_t e = cudaFuncSetAttribute(syrk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM);
       if (e != cudaSuccess) return e;
-      attr = true;
+      attr.fetch_or(bit);
     }
     SyrkParams p;
     p.N = N; p.n = n; p.nblk = pl.nblk; p.npairs = pl.npairs; p.nslices = pl.nslices;

@@ -746,13 +746,18 @@ struct HinvGraph {
 
 cudaError_t launch_hinv(const double* H, int64_t n, double alpha, double* h, double* ws, DevStatus* st,
                         cudaStream_t s) {
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaFuncSetAttribute(pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPpSmem);
-    cudaFuncSetAttribute(trail_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(2 * kTileBytes));
-    cudaFuncSetAttribute(rowmult_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(2 * kTileBytes));
-    cudaFuncSetAttribute(inv_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(2 * kTileBytes));
-    attr_done = true;
+  static std::atomic<uint64_t> attr{0};
+  uint64_t bit = 0;
+  if (attr_pending(attr, bit)) {
+    cudaError_t e = cudaFuncSetAttribute(pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPpSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(trail_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(2 * kTileBytes));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(rowmult_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(2 * kTileBytes));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(inv_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(2 * kTileBytes));
+    if (e != cudaSuccess) return e;
+    attr.fetch_or(bit);
   }
   const int T = (int)((pad32(n) + NB - 1) / NB);
   HinvStreams& hs = hinv_streams(2 * T + 6);

@@ -814,12 +814,13 @@ static cudaError_t launch_score(const SbaPlan& pl, int64_t m, int64_t n, int64_t
   p.N = N; p.m = m; p.n = n; p.g = group; p.k = pl.k; p.P = pl.P; p.ksplit = pl.ksplit;
   p.n_tt = pl.n_tt; p.n_tp = tp1 - tp0; p.n_ot = pl.n_ot; p.stages = pl.stages; p.nA = pl.nA; p.nD = pl.nD;
   p.order = order; p.part = reinterpret_cast<float*>(sw); p.yd = yd; p.tp0 = tp0; p.st = st;
-  static bool attr = false;
-  if (!attr) {  // the plan's shared memory never exceeds this bound
+  static std::atomic<uint64_t> attr{0};
+  uint64_t bit = 0;
+  if (attr_pending(attr, bit)) {  // the plan's shared memory never exceeds this bound
     cudaError_t e = cudaFuncSetAttribute(sba_score_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          227 * 1024);
     if (e != cudaSuccess) return e;
-    attr = true;
+    attr.fetch_or(bit);
   }
   const int units = p.n_tp * pl.n_ot;
   const int grid = units < num_sms ? units : num_sms;
