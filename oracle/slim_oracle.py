@@ -278,16 +278,18 @@ def sba_search(W: np.ndarray, X: ArrayOrChunks, order: Sequence[int], group: int
             for p in range(P):
                 kl_sum[p] += kl_per_token(Y, x @ dequant(p).T).sum()
         else:
-            prev = dequant(0)
-            Yq = x @ prev.T
+            Yq = x @ dequant(0).T
             kl_sum[0] += kl_per_token(Y, Yq).sum()
             for p in range(1, P):
-                cur = dequant(p)
                 for c in (order[p - 1], order[k - p]):
+                    # candidates p-1 and p differ only on group c; the quantizer
+                    # is per group, so its block quantized at either bit width is
+                    # what the whole-matrix dequantization would hold there
                     cols = slice(c * group, (c + 1) * group)
-                    Yq = Yq + x[:, cols] @ (cur[:, cols] - prev[:, cols]).T
+                    blk = W[:, cols]
+                    d = rtn_dequant(blk, [allocs[p][c]], group) - rtn_dequant(blk, [allocs[p - 1][c]], group)
+                    Yq = Yq + x[:, cols] @ d.T
                 kl_sum[p] += kl_per_token(Y, Yq).sum()
-                prev = cur
     kl = kl_sum / ntok
     p_star = int(np.argmin(kl))
     srt = np.sort(kl)
