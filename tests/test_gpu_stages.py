@@ -85,6 +85,25 @@ def test_hinv_not_positive_definite():
     with pytest.raises(slim.SlimError) as e:
         slim.slim_hinv_diag(torch.from_numpy(H).cuda(), 0.0)
     assert e.value.status == 5
+    assert e.value.device_detail == 0          # the first pivot fails
+
+
+def test_hinv_not_positive_definite_reports_the_pivot():
+    """A positive definite matrix with one bad pivot deep inside (column 150 of 320:
+    block 2, sub-block 1): the reported index is that column."""
+    n, bad = 320, 150
+    rng = np.random.default_rng(4)
+    X = rng.standard_normal((4 * n, n))
+    H = O.hessian(X)
+    H[bad, :] = 0.0
+    H[:, bad] = 0.0
+    H[bad, bad] = -1.0          # a negative diagonal entry with its row and column cleared
+    with pytest.raises(slim.SlimError) as e:
+        slim.slim_hinv_diag(torch.from_numpy(H).cuda(), 0.0)
+    assert e.value.status == 5
+    assert e.value.device_detail == bad
+    ok = slim.slim_hinv_diag(torch.from_numpy(O.hessian(X)).cuda(), 0.01)   # the next call succeeds
+    assert torch.isfinite(ok).all()
 
 
 # ---------------------------------------------------------------- salience
