@@ -666,11 +666,17 @@ __global__ void sba_final_kernel(const double* __restrict__ kl_part, int n_tt, i
                                  int32_t* __restrict__ pstar_out, uint8_t* __restrict__ bits) {
   __shared__ double s_kl[SB_MAX_K / 2 + 1];
   __shared__ int s_p;
-  for (int q = threadIdx.x; q < P; q += blockDim.x) {
+  // one warp per candidate: lane l adds token tiles l, l + 32, ... in order,
+  // then a fixed shuffle tree (the same order every run)
+  const int lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int q = threadIdx.x >> 5; q < P; q += nw) {
     double acc = 0.0;
-    for (int t = 0; t < n_tt; ++t) acc += kl_part[(size_t)q * n_tt + t];
-    s_kl[q] = acc / (double)N;
-    if (kl_out) kl_out[q] = s_kl[q];
+    for (int t = lane; t < n_tt; t += 32) acc += kl_part[(size_t)q * n_tt + t];
+    acc = warp_sum(acc);
+    if (lane == 0) {
+      s_kl[q] = acc / (double)N;
+      if (kl_out) kl_out[q] = s_kl[q];
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0) {
