@@ -66,3 +66,30 @@ def test_stage_argument_validation(lib):
     assert lib.slim_hinv_diag(0x1000, 64, -1.0, 0x2000, None, 0, None) == 1      # negative damping
     assert lib.slim_salience(0x1000, 8, 256, 0x2000, 64, None, 0x3000, None, 0, None) == 1  # NULL S
     assert lib.slim_sqc(0x1000, 8, 256, 0x2000, 0x3000, 128, 2, 0.1, 0, 1, 2, 3, None, None) == 1
+
+
+@pytest.mark.parametrize("m, n, N, xdtype, group", [
+    (4096, 4096, 262144, 1, 128), (4096, 11008, 262144, 1, 128), (13824, 5120, 262144, 1, 32),
+    (256, 512, 2048, 0, 128), (300, 640, 5000, 1, 64)])
+def test_workspace_sizes(lib, m, n, N, xdtype, group):
+    """Workspace sizes are pure host arithmetic: the split search needs the one-pass
+    search's workspace plus its stored phase-A state (8 bytes per token tile row and
+    output column, tiles padded to 128), and the whole layer holds H and the SBA
+    operands at least."""
+    one = lib.slim_sba_workspace_bytes(m, n, N, xdtype, group)
+    split = lib.slim_sba_split_workspace_bytes(m, n, N, xdtype, group)
+    tiles_t, tiles_o = -(-N // 128), -(-m // 128)
+    assert split >= one + tiles_t * tiles_o * 128 * 128 * 8
+    assert split - one <= tiles_t * tiles_o * 128 * 128 * 8 + 512
+    ksplit = 1 if xdtype == 1 else 2
+    operands = 4 * m * n * 2 + N * n * 2 * ksplit                   # three RTN arrays, W, X as fp16
+    assert one >= operands
+    layer = lib.slim_workspace_bytes(m, n, N, xdtype, group, 2)
+    assert layer >= n * n * 8 + operands
+
+
+def test_split_search_rejects_bad_chunks_before_any_launch(lib):
+    for chunk in (0, -256, 100, 384):
+        rc = lib.slim_sba_search_split(0x1000, 256, 512, 0x2000, 1, 4096, 128, 2, 0x3000, None, None, 0x4000, chunk,
+                                       None, 0, None)
+        assert rc == 1, chunk
