@@ -632,7 +632,8 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
 __global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict__ part, int n_ot, int P, int64_t N,
                                                         int n_tt, double* __restrict__ kl_part) {
   extern __shared__ float s_f[];  // [n_ot][128] scale factors (one partial set per output tile)
-  __shared__ double red[4];
+  constexpr int QB = 8;  // candidates per pass
+  __shared__ double red[4][QB];
   const int tt = blockIdx.x, r = threadIdx.x;
   const int F = 2 + 2 * P;
   const bool valid = (int64_t)tt * SB_BM + r < N;
@@ -645,18 +646,33 @@ __global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict_
     s_f[og * SB_BM + r] = f;
     Sy += (double)base[(size_t)og * F * SB_BM + SB_BM] * (double)f;
   }
-  for (int q = 0; q < P; ++q) {
-    double sq = 0.0, a = 0.0;
+  // candidates in blocks of QB: one pass over the output tiles loads 2 QB
+  // independent values per tile (the sums run over the tiles in order, as
+  // one candidate at a time would)
+  for (int q0 = 0; q0 < P; q0 += QB) {
+    const int nq = (P - q0 < QB) ? P - q0 : QB;
+    double sq[QB], a[QB];
+#pragma unroll
+    for (int j = 0; j < QB; ++j) sq[j] = a[j] = 0.0;
     for (int og = 0; og < n_ot; ++og) {
       const double f = s_f[og * SB_BM + r];
-      sq += (double)base[((size_t)og * F + 2 + 2 * q) * SB_BM] * f;
-      a += (double)base[((size_t)og * F + 3 + 2 * q) * SB_BM] * f;
+      const float* bq = base + ((size_t)og * F + 2 + 2 * q0) * SB_BM;
+#pragma unroll
+      for (int j = 0; j < QB; ++j)
+        if (j < nq) {
+          sq[j] += (double)bq[(size_t)(2 * j) * SB_BM] * f;
+          a[j] += (double)bq[(size_t)(2 * j + 1) * SB_BM] * f;
+        }
     }
-    double kl = valid ? (log(sq / Sy) - a / Sy) : 0.0;
-    kl = warp_sum(kl);
-    if ((r & 31) == 0) red[r >> 5] = kl;
+#pragma unroll
+    for (int j = 0; j < QB; ++j)
+      if (j < nq) {
+        double kl = valid ? (log(sq[j] / Sy) - a[j] / Sy) : 0.0;
+        kl = warp_sum(kl);
+        if ((r & 31) == 0) red[r >> 5][j] = kl;
+      }
     __syncthreads();
-    if (r == 0) kl_part[(size_t)q * n_tt + tt] = (red[0] + red[1]) + (red[2] + red[3]);
+    if (r < nq) kl_part[(size_t)(q0 + r) * n_tt + tt] = (red[0][r] + red[1][r]) + (red[2][r] + red[3][r]);
     __syncthreads();
   }
 }
