@@ -220,6 +220,8 @@ def slim_sba_search(W: torch.Tensor, X: torch.Tensor, group: int, avg_bits: int,
 
 def slim_sba_search_split(W: torch.Tensor, X: torch.Tensor, group: int, avg_bits: int, order: torch.Tensor,
                           chunk_tokens: int, ws=None, stream=None):
+    """slim_sba_search's outputs from the two-part schedule: phase A per chunk of
+    chunk_tokens tokens (a multiple of 256), then the candidate steps."""
     m, n = W.shape
     N = X.shape[0]
     k = n // group
