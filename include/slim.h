@@ -18,8 +18,12 @@
  *   or 128 and must divide n. avg_bits is the average bit-width b (2..7); the
  *   groups get b-1, b or b+1 bits.
  * - Every array argument is DEVICE memory owned by the caller unless marked
- *   HOST. The library keeps no state between calls and never frees caller
- *   memory. Arrays must not overlap. W must be 16-byte aligned and X too.
+ *   HOST. The library keeps no data between calls and never frees caller
+ *   memory; it caches, per host thread and device, a few CUDA streams and
+ *   events and the inverse stage's CUDA graph (created on first use, kept
+ *   until the process exits). Work on those side streams is ordered after
+ *   `stream` and joined back into it before the call returns. Arrays must
+ *   not overlap. W must be 16-byte aligned and X too.
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *   Work is ordered on it. Each call enqueues its kernels, then waits for the
  *   stream to drain and reads the call's device status word, so that it can
