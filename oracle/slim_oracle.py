@@ -214,16 +214,23 @@ def log_softmax(Z: np.ndarray) -> np.ndarray:
     return Z - mx - np.log(np.exp(Z - mx).sum(axis=1, keepdims=True))
 
 
-def kl_per_token(Y: np.ndarray, Yq: np.ndarray) -> np.ndarray:
+def kl_per_token(Y: np.ndarray, Yq: np.ndarray, ref=None) -> np.ndarray:
     """KL(softmax(y_t) || softmax(yq_t)) for every token t (row).
 
     [P1 组件一 SBA] scores an allocation by the KL divergence of the layer
     outputs. Reading: softmax over the output features, direction
-    KL(full precision || quantized).
+    KL(full precision || quantized). `ref` may carry (log_softmax(Y), its
+    exp) computed once for several Yq against the same Y: the same values.
     """
-    lp = log_softmax(Y)
+    lp, p = ref if ref is not None else kl_reference(Y)
     lq = log_softmax(Yq)
-    return np.sum(np.exp(lp) * (lp - lq), axis=1)
+    return np.sum(p * (lp - lq), axis=1)
+
+
+def kl_reference(Y: np.ndarray):
+    """log_softmax(Y) and softmax(Y) = exp(log_softmax(Y)), the full-precision side of kl_per_token."""
+    lp = log_softmax(Y)
+    return lp, np.exp(lp)
 
 
 # ---------------------------------------------------------------------------
@@ -278,8 +285,9 @@ def sba_search(W: np.ndarray, X: ArrayOrChunks, order: Sequence[int], group: int
             for p in range(P):
                 kl_sum[p] += kl_per_token(Y, x @ dequant(p).T).sum()
         else:
+            ref = kl_reference(Y)   # the same for every candidate of this chunk
             Yq = x @ dequant(0).T
-            kl_sum[0] += kl_per_token(Y, Yq).sum()
+            kl_sum[0] += kl_per_token(Y, Yq, ref).sum()
             for p in range(1, P):
                 for c in (order[p - 1], order[k - p]):
                     # candidates p-1 and p differ only on group c; the quantizer
@@ -289,7 +297,7 @@ def sba_search(W: np.ndarray, X: ArrayOrChunks, order: Sequence[int], group: int
                     blk = W[:, cols]
                     d = rtn_dequant(blk, [allocs[p][c]], group) - rtn_dequant(blk, [allocs[p - 1][c]], group)
                     Yq = Yq + x[:, cols] @ d.T
-                kl_sum[p] += kl_per_token(Y, Yq).sum()
+                kl_sum[p] += kl_per_token(Y, Yq, ref).sum()
     kl = kl_sum / ntok
     p_star = int(np.argmin(kl))
     srt = np.sort(kl)
