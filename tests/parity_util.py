@@ -94,3 +94,37 @@ def compare_sqc(words_gpu, scale_gpu, zero_gpu, tau_gpu, ref: O.SQCResult, bits,
 def balanced_bits(k, avg_bits, p, seed):
     rng = np.random.default_rng(seed)
     return O.allocation(rng.permutation(k), avg_bits, p).astype(np.uint8)
+
+
+def comparable_candidates(order_gpu, order_ref):
+    """Candidates p whose promoted and demoted group sets are the same under both orders
+    (the score of a candidate depends only on those two sets)."""
+    a, b = np.asarray(order_gpu), np.asarray(order_ref)
+    k = a.size
+    return [p for p in range(k // 2 + 1)
+            if set(a[:p].tolist()) == set(b[:p].tolist()) and set(a[k - p:].tolist()) == set(b[k - p:].tolist())]
+
+
+def allocation_ok(bits_gpu, order_gpu, p_gpu, bits_ref, kl_ref, S_ref, avg_bits, kl_tol=2 * KL_ATOL, s_rel=1e-5):
+    """The GPU's allocation against the stored one. It must be the allocation its own order
+    and p* define, and equal the stored one except where the stored values are near ties that
+    the GPU's arithmetic can resolve either way: a p* whose stored KL is within kl_tol of the
+    best, or groups swapped across a promote/demote boundary whose stored saliences differ by
+    less than s_rel. Returns '' when equal, else what differed."""
+    bits_gpu = np.asarray(bits_gpu).astype(int)
+    bits_ref = np.asarray(bits_ref).astype(int)
+    kl_ref = np.asarray(kl_ref, dtype=np.float64)
+    S_ref = np.asarray(S_ref, dtype=np.float64)
+    assert bits_gpu.tolist() == O.allocation(np.asarray(order_gpu), avg_bits, p_gpu).tolist()
+    p_ref = int(np.argmin(kl_ref))
+    if p_gpu != p_ref:
+        gap = kl_ref[p_gpu] - kl_ref[p_ref]
+        assert gap <= kl_tol, f"p* {p_gpu} vs stored {p_ref}: stored KL gap {gap:.3e}"
+        return "p* (near tie)"
+    if (bits_gpu == bits_ref).all():
+        return ""
+    diff = np.nonzero(bits_gpu != bits_ref)[0]
+    for c in diff:
+        near = [o for o in diff if o != c and abs(S_ref[c] - S_ref[o]) <= s_rel * max(abs(S_ref[c]), abs(S_ref[o]))]
+        assert near, f"group {c} has bits {bits_gpu[c]} vs stored {bits_ref[c]} with no near-tie partner"
+    return "near-tie swap"

@@ -15,7 +15,8 @@ from post_weight_quantization_hessian_b200 import synthetic as syn
 import json
 import os
 
-from parity_util import KL_ATOL, compare_sqc, device_inputs, hessian_bound, order_ok, pstar_ok, x_f64
+from parity_util import (KL_ATOL, allocation_ok, comparable_candidates, compare_sqc, device_inputs, hessian_bound,
+                         order_ok, pstar_ok, x_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -133,11 +134,16 @@ def test_full_size_sampled(workload):
     # S inherit about twice that relative shift, nearly uniform across groups
     np.testing.assert_allclose(g["S"], S_gold, rtol=2 * hessian_bound(s.N))
     mism = order_ok(g["order"], S_gold, rel=1e-5)
-    assert np.abs(g["kl"] - np.array(gold["kl"])).max() <= KL_ATOL
-    assert g["p_star"] == gold["p_star"]
-    assert g["bits"].astype(int).tolist() == gold["bits"]
-    print(f"full-size vs golden: order mismatches {mism} (near ties only), max |dKL| "
-          f"{np.abs(g['kl'] - np.array(gold['kl'])).max():.2e}, p* {g['p_star']}")
+    # KL of the candidates whose promoted and demoted sets agree under both orders (all
+    # of them unless a near tie swapped two groups), then the allocation itself
+    comp = comparable_candidates(g["order"], gold["order"])
+    kl_gold = np.array(gold["kl"])
+    dkl = np.abs(np.asarray(g["kl"])[comp] - kl_gold[comp]).max()
+    assert dkl <= KL_ATOL
+    how = allocation_ok(g["bits"], g["order"], int(g["p_star"]), gold["bits"], kl_gold, S_gold, s.avg_bits)
+    print(f"full-size vs golden: order mismatches {mism} (near ties only), {len(comp)} of {len(kl_gold)} "
+          f"candidates comparable, max |dKL| {dkl:.2e}, p* {g['p_star']} vs {gold['p_star']}, "
+          f"allocation {how or 'equal'}")
     # full-N search: invariants
     kl = g["kl"]
     assert np.all(kl >= 0) and g["p_star"] == int(np.argmin(kl))
