@@ -1,6 +1,6 @@
 """Write oracle decisions for a full-size workload to tests/golden/<name>.json.
 
-    python tests/golden/make_golden.py [--workload llama7b_q_proj_4096x4096] [--procs 8]
+    python tests/golden/make_golden.py [--workload llama7b_q_proj_4096x4096] [--procs 8] [--out-dir DIR]
 
 Everything stored comes from oracle/ (float64 CPU) on the seeded synthetic
 inputs: group salience S, the order and its consecutive relative gaps, the
@@ -53,6 +53,8 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="llama7b_q_proj_4096x4096")
     ap.add_argument("--procs", type=int, default=os.cpu_count())
+    ap.add_argument("--out-dir", default=os.path.dirname(os.path.abspath(__file__)),
+                    help="where to write <workload>.json (default: beside this script)")
     a = ap.parse_args(argv)
     from oracle import slim_oracle as O
     from post_weight_quantization_hessian_b200 import synthetic as syn
@@ -90,7 +92,7 @@ def main(argv=None):
         "bits": O.allocation(order, spec.avg_bits, p_star).tolist(),
         "seconds": {"hessian": t_h - t0, "hinv_salience": t_s - t_h, "sba": time.time() - t_s},
     }
-    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), f"{a.workload}.json")
+    path = os.path.join(a.out_dir, f"{a.workload}.json")
     with open(path, "w") as f:
         json.dump(out, f, indent=1)
     print(json.dumps({k: out[k] for k in ("order", "p_star", "kl_margin", "seconds")}))
