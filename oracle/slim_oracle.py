@@ -253,8 +253,18 @@ def sba_candidates(k: int) -> int:
     return k // 2 + 1
 
 
+def mse_per_token(Y: np.ndarray, Yq: np.ndarray) -> np.ndarray:
+    """Mean over the output features of (yq_t - y_t)^2 for every token t (row).
+
+    The objective SBA's KL is compared against in the method's ablation
+    [P2 Measured effects: KL divergence rather than MSE as the SBA objective].
+    """
+    D = np.asarray(Yq, dtype=np.float64) - np.asarray(Y, dtype=np.float64)
+    return np.mean(D * D, axis=1)
+
+
 def sba_search(W: np.ndarray, X: ArrayOrChunks, order: Sequence[int], group: int, avg_bits: int,
-               reassociate: bool = False) -> SBAResult:
+               reassociate: bool = False, objective: str = "kl") -> SBAResult:
     """Pick p* = argmin_p mean_t KL(softmax(x_t W^T) || softmax(x_t W_p^T)).
 
     [P1 组件一 SBA], [P2 Approach]: candidates are the balanced allocations
@@ -262,9 +272,16 @@ def sba_search(W: np.ndarray, X: ArrayOrChunks, order: Sequence[int], group: int
     Every p in [0, k/2] is scored (the double-pointer walk visits them all), and
     the smallest p reaching the least KL wins.
 
+    `objective="mse"` scores a candidate by mse_per_token instead (the ablation
+    of [P2 Measured effects]). `order` may be any permutation of the groups:
+    the salience order is the method; position order (head-tail) and a random
+    permutation are the allocations of the ablation [P1 Fig. 5 caption].
+
     `reassociate=True` computes X W_p^T as X W_{p-1}^T plus the product of the
     two changed column groups, which is the same sum regrouped.
     """
+    if objective not in ("kl", "mse"):
+        raise ValueError("objective must be 'kl' or 'mse'")
     W = np.asarray(W, dtype=np.float64)
     k = W.shape[1] // group
     P = sba_candidates(k)
@@ -283,11 +300,13 @@ def sba_search(W: np.ndarray, X: ArrayOrChunks, order: Sequence[int], group: int
         ntok += x.shape[0]
         if not reassociate:
             for p in range(P):
-                kl_sum[p] += kl_per_token(Y, x @ dequant(p).T).sum()
+                Yq = x @ dequant(p).T
+                kl_sum[p] += (kl_per_token(Y, Yq) if objective == "kl" else mse_per_token(Y, Yq)).sum()
         else:
-            ref = kl_reference(Y)   # the same for every candidate of this chunk
+            ref = kl_reference(Y) if objective == "kl" else None   # the same for every candidate of this chunk
+            score = (lambda Yq: kl_per_token(Y, Yq, ref)) if objective == "kl" else (lambda Yq: mse_per_token(Y, Yq))
             Yq = x @ dequant(0).T
-            kl_sum[0] += kl_per_token(Y, Yq, ref).sum()
+            kl_sum[0] += score(Yq).sum()
             for p in range(1, P):
                 for c in (order[p - 1], order[k - p]):
                     # candidates p-1 and p differ only on group c; the quantizer
@@ -297,7 +316,7 @@ def sba_search(W: np.ndarray, X: ArrayOrChunks, order: Sequence[int], group: int
                     blk = W[:, cols]
                     d = rtn_dequant(blk, [allocs[p][c]], group) - rtn_dequant(blk, [allocs[p - 1][c]], group)
                     Yq = Yq + x[:, cols] @ d.T
-                kl_sum[p] += kl_per_token(Y, Yq, ref).sum()
+                kl_sum[p] += score(Yq).sum()
     kl = kl_sum / ntok
     p_star = int(np.argmin(kl))
     srt = np.sort(kl)

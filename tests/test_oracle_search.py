@@ -117,3 +117,61 @@ def test_kl_nonnegative_and_high_bits_small():
     assert np.all(lo >= 0) and np.all(hi >= 0)
     # small-noise KL grows with the output noise variance; 5 more bits divide it by about 4^5
     assert 0.25 / 1024 < hi[0] / lo[0] < 4.0 / 1024
+
+
+def test_mse_objective_closed_form_through_the_hessian():
+    """MSE_p = mean over tokens and outputs of (x (W_p - W)^T)^2
+    = trace(E_p (X^T X) E_p^T) / (N m) with E_p = W_p - W: the same number from
+    the Gram matrix, without forming any layer output."""
+    W, X = small_layer(seed=3)
+    g, k = 8, 6
+    m, N = W.shape[0], X.shape[0]
+    S = O.group_salience(W, O.hinv_diag(O.hessian(X)), g)
+    order = O.salience_order(S)
+    G = X.T @ X
+    for reassociate in (False, True):
+        r = O.sba_search(W, X, order, g, 2, reassociate=reassociate, objective="mse")
+        for p in range(k // 2 + 1):
+            E = O.rtn_dequant(W, O.allocation(order, 2, p), g) - W
+            assert r.kl[p] == pytest.approx(np.trace(E @ G @ E.T) / (N * m), rel=1e-10)
+        assert r.p_star == int(np.argmin(r.kl))
+
+
+def test_mse_objective_brute_force_and_bit_growth():
+    """Every balanced allocation scored by hand: the search's MSE equals the
+    brute-force value for the salience-ordered ones; raising every group's
+    bits lowers the error about 4x per bit."""
+    W, X = small_layer(seed=4)
+    g, k = 8, 6
+    order = O.salience_order(O.group_salience(W, O.hinv_diag(O.hessian(X)), g))
+    r = O.sba_search(W, X, order, g, 2, objective="mse")
+    Y = X @ W.T
+    for p in range(k // 2 + 1):
+        Yq = X @ O.rtn_dequant(W, O.allocation(order, 2, p), g).T
+        assert r.kl[p] == pytest.approx(np.mean((Yq - Y) ** 2), rel=1e-12)
+    e = [np.mean((X @ O.rtn_dequant(W, [b] * k, g).T - Y) ** 2) for b in (3, 4, 5, 6)]
+    ratios = np.array(e[:-1]) / np.array(e[1:])
+    assert np.all((ratios > 2.5) & (ratios < 6.5))
+
+
+@pytest.mark.parametrize("kind", ["head_tail", "random"])
+def test_search_with_a_given_order(kind):
+    """Head-tail (groups in position order) and random allocation: the search
+    promotes order[:p] and demotes order[k-p:] of the order it is given, and
+    its scores equal the brute-force scores of those allocations."""
+    W, X = small_layer(seed=5)
+    g, k = 8, 6
+    order = np.arange(k) if kind == "head_tail" else np.random.default_rng(9).permutation(k)
+    for objective in ("kl", "mse"):
+        r = O.sba_search(W, X, order, g, 2, objective=objective)
+        Y = X @ W.T
+        for p in range(k // 2 + 1):
+            bits = np.full(k, 2)
+            bits[order[:p]] = 3
+            if p:
+                bits[order[k - p:]] = 1
+            Yq = X @ O.rtn_dequant(W, bits, g).T
+            ref = (np.mean([entropy(softmax(Y[t]), softmax(Yq[t])) for t in range(X.shape[0])])
+                   if objective == "kl" else np.mean((Yq - Y) ** 2))
+            assert r.kl[p] == pytest.approx(ref, rel=1e-10)
+        assert r.bits.tolist() == O.allocation(order, 2, r.p_star).tolist()
