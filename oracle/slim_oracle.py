@@ -386,6 +386,37 @@ class SQCResult:
     mask_rate: float        # fraction of weights in the 3-sigma masks
 
 
+def sqc_group(w: np.ndarray, h: np.ndarray, b: int, lam: float, n_tau: int):
+    """SQC for one group of columns: w is [rows, g], h the g inverse-Hessian entries.
+
+    Returns (codes [rows, g], s [rows], z [rows], t* [rows], margin [rows],
+    masked count). The per-row steps are those of sqc_calibrate below.
+    """
+    taus = tau_grid(lam, n_tau)
+    m = w.shape[0]
+    delta = element_salience(w, h)
+    mask = salient_mask(w)
+    lo, hi, s0, z0, deg = minmax_params(w, b)
+    errs = np.empty((m, n_tau))
+    for t, tau in enumerate(taus):
+        s = tau * s0
+        _, wq = fake_quant(w, s, z0, b)
+        errs[:, t] = sqc_error(w, delta, mask, wq)
+    best = np.argmin(errs, axis=1)
+    best[deg] = 0
+    s_best = taus[best] * s0
+    s_best[deg] = 1.0
+    q, _ = fake_quant(w, s_best, z0, b)
+    q[deg] = 0.0
+    margin = np.full(m, np.inf)
+    if n_tau > 1:
+        srt = np.sort(errs, axis=1)
+        gap = (srt[:, 1] - srt[:, 0]) / np.maximum(srt[:, 0], 1e-300)
+        gap[deg] = np.inf
+        margin = gap
+    return q.astype(np.int64), s_best, np.asarray(z0, dtype=np.float64), best, margin, int(mask.sum())
+
+
 def sqc_calibrate(W: np.ndarray, h: np.ndarray, bits: Sequence[int], group: int, lam: float,
                   n_tau: int) -> SQCResult:
     """Per (row, group): 3-sigma mask, then the tau with least weighted error.
@@ -400,7 +431,6 @@ def sqc_calibrate(W: np.ndarray, h: np.ndarray, bits: Sequence[int], group: int,
     h = np.asarray(h, dtype=np.float64)
     m, n = W.shape
     k = n // group
-    taus = tau_grid(lam, n_tau)
     codes = np.zeros((m, n), dtype=np.int64)
     scale64 = np.zeros((m, k))
     zero64 = np.zeros((m, k))
@@ -408,33 +438,14 @@ def sqc_calibrate(W: np.ndarray, h: np.ndarray, bits: Sequence[int], group: int,
     margin = np.full((m, k), np.inf)
     masked = 0
     for c in range(k):
-        b = int(bits[c])
         cols = slice(c * group, (c + 1) * group)
-        w = W[:, cols]
-        delta = element_salience(w, h[cols])
-        mask = salient_mask(w)
-        masked += int(mask.sum())
-        lo, hi, s0, z0, deg = minmax_params(w, b)
-        errs = np.empty((m, n_tau))
-        for t, tau in enumerate(taus):
-            s = tau * s0
-            _, wq = fake_quant(w, s, z0, b)
-            errs[:, t] = sqc_error(w, delta, mask, wq)
-        best = np.argmin(errs, axis=1)
-        best[deg] = 0
-        s_best = taus[best] * s0
-        s_best[deg] = 1.0
-        q, _ = fake_quant(w, s_best, z0, b)
-        q[deg] = 0.0
-        codes[:, cols] = q.astype(np.int64)
+        q, s_best, z0, best, mg, nm = sqc_group(W[:, cols], h[cols], int(bits[c]), lam, n_tau)
+        masked += nm
+        codes[:, cols] = q
         scale64[:, c] = s_best
         zero64[:, c] = z0
         tidx[:, c] = best
-        if n_tau > 1:
-            srt = np.sort(errs, axis=1)
-            gap = (srt[:, 1] - srt[:, 0]) / np.maximum(srt[:, 0], 1e-300)
-            gap[deg] = np.inf
-            margin[:, c] = gap
+        margin[:, c] = mg
     return SQCResult(codes=codes, scale=scale64.astype(np.float32), zero=zero64.astype(np.float32),
                      tau_idx=tidx, scale64=scale64, zero64=zero64, margin=margin,
                      mask_rate=masked / float(m * n))
@@ -445,6 +456,85 @@ def dequant_codes(codes: np.ndarray, scale: np.ndarray, zero: np.ndarray, group:
     s = np.repeat(np.asarray(scale, dtype=np.float64), group, axis=1)
     z = np.repeat(np.asarray(zero, dtype=np.float64), group, axis=1)
     return s * (np.asarray(codes, dtype=np.float64) - z)
+
+
+# ---------------------------------------------------------------------------
+# GPTQ backbone: column-by-column quantization with error compensation
+# ---------------------------------------------------------------------------
+def gptq_factor(H: np.ndarray, alpha: float = DAMP_ALPHA):
+    """U upper triangular with H_d^-1 = U^T U (the Cholesky factor of the damped
+    inverse Hessian), and the diagonal of H_d^-1.
+
+    GPTQ's compensation uses the rows of U; H_d is the damped Hessian of the
+    rest of the path (dead columns set to 1, then alpha * mean diagonal).
+    """
+    Hd = damped(H, alpha)
+    try:
+        Hinv = np.linalg.inv(Hd)
+        U = np.linalg.cholesky(Hinv).T
+    except np.linalg.LinAlgError as e:
+        raise NotPositiveDefinite(str(e)) from e
+    return U, np.diagonal(Hinv).copy()
+
+
+@dataclass
+class GPTQResult:
+    codes: np.ndarray       # [m, n] integer codes
+    scale: np.ndarray       # [m, k] float32
+    zero: np.ndarray        # [m, k] float32
+    tau_idx: np.ndarray     # [m, k] chosen tau index
+    scale64: np.ndarray
+    zero64: np.ndarray
+    margin: np.ndarray      # [m, k] SQC's relative gap best -> second best error
+    Wq: np.ndarray          # [m, n] float64 dequantized weights
+    h: np.ndarray           # [n] diag of the damped inverse Hessian
+    snapshot: Optional[np.ndarray] = None
+
+
+def gptq_quantize(W: np.ndarray, H: np.ndarray, bits: Sequence[int], group: int, lam: float, n_tau: int,
+                  alpha: float = DAMP_ALPHA, snapshot_after: Optional[int] = None) -> GPTQResult:
+    """SliM-LLM inside the GPTQ layer loop [P1 核心设计: the GPTQ layer-wise
+    quantization skeleton with the two salience-driven components inserted; P1
+    FAQ]: columns are quantized in order; when a group's first column is
+    reached, SQC calibrates the group's quantizer (bits from SBA, 3-sigma mask,
+    tau search) on the group's weights as the earlier columns' compensation has
+    left them; each column is then rounded with its group's quantizer and its
+    error, divided by U_jj, is spread over the later columns along row j of U.
+
+    Readings (the pages name GPTQ but do not restate it): columns in their
+    natural order (no reordering by activation size); a group's scale and zero
+    are fixed when its first column is reached; the element salience inside SQC
+    uses the current weights and diag(H_d^-1); dead columns only get H_jj = 1.
+    `snapshot_after=j` also returns the working weights right after column j.
+    """
+    W = np.asarray(W, dtype=np.float64)
+    m, n = W.shape
+    k = n // group
+    U, hd = gptq_factor(H, alpha)
+    Wk = W.copy()
+    codes = np.zeros((m, n), dtype=np.int64)
+    Wq = np.zeros((m, n))
+    scale64 = np.zeros((m, k))
+    zero64 = np.zeros((m, k))
+    tidx = np.zeros((m, k), dtype=np.int64)
+    margin = np.full((m, k), np.inf)
+    snap = None
+    for j in range(n):
+        c = j // group
+        b = int(bits[c])
+        if j % group == 0:
+            cols = slice(c * group, (c + 1) * group)
+            _, s_c, z_c, t_c, mg, _ = sqc_group(Wk[:, cols], hd[cols], b, lam, n_tau)
+            scale64[:, c], zero64[:, c], tidx[:, c], margin[:, c] = s_c, z_c, t_c, mg
+        q, wq = fake_quant(Wk[:, j:j + 1], scale64[:, c], zero64[:, c], b)
+        codes[:, j] = q[:, 0].astype(np.int64)
+        Wq[:, j] = wq[:, 0]
+        err = (Wk[:, j] - wq[:, 0]) / U[j, j]
+        Wk[:, j + 1:] -= np.outer(err, U[j, j + 1:])
+        if snapshot_after == j:
+            snap = Wk.copy()
+    return GPTQResult(codes=codes, scale=scale64.astype(np.float32), zero=zero64.astype(np.float32), tau_idx=tidx,
+                      scale64=scale64, zero64=zero64, margin=margin, Wq=Wq, h=hd, snapshot=snap)
 
 
 # ---------------------------------------------------------------------------
