@@ -31,7 +31,14 @@
  *   complete when the call returns SLIM_OK.
  * - Workspace: `ws` is device scratch of at least the size the matching
  *   *_workspace_bytes function returns, 256-byte aligned. ws == NULL makes the
- *   call allocate (cudaMallocAsync on `stream`) and free it itself.
+ *   call allocate it (cudaMallocFromPoolAsync on `stream`) and free it itself,
+ *   from a memory pool the library creates per device on first use and keeps
+ *   until the process exits (freed blocks stay in that pool for the next call).
+ *   The device's default pool and its settings are not touched.
+ * - Per-device state (the pool, cached streams, events and graphs, the address
+ *   of slim_salience_noalloc's array) is created on first use on a device; a
+ *   cudaDeviceReset of that device invalidates it, so a process that resets a
+ *   device must not call the library on that device again.
  * - Errors are returned, never raised: on any status other than SLIM_OK the
  *   outputs are unspecified. Arguments are validated before any launch.
  * - Calls on the same device that share a workspace must not overlap.
@@ -61,6 +68,24 @@ typedef enum {
 
 typedef enum { SLIM_X_F32 = 0, SLIM_X_BF16 = 1 } slim_xdtype;
 
+/* How SBA scores a candidate allocation. SLIM_OBJ_KL is the method's
+ * objective ([P1] 组件一 SBA: output KL divergence). SLIM_OBJ_MSE, the mean
+ * squared error of the layer outputs, is the objective the method is compared
+ * against in its ablation ([P2] Measured effects: KL rather than MSE). */
+typedef enum { SLIM_OBJ_KL = 0, SLIM_OBJ_MSE = 1 } slim_objective;
+
+/* Operand precision of the SBA scoring's weight side (bf16 X). Each 64-column
+ * box of the weight-side arrays is an fp16 value (11 significant bits) or an
+ * fp16 hi/lo pair (22 bits, twice the tensor-core work on that box).
+ * SLIM_SBA_ADAPTIVE pairs the boxes that carry the most output rounding error:
+ * per box the estimate sum_j |x_j|^2 |w_j|^2 (column energies of W and of the
+ * first 16384 tokens of X) is ranked, and boxes are paired in descending order
+ * until at most 1/32 of the total estimate is left; with activation-outlier
+ * channels that is typically the few boxes holding them. SLIM_SBA_FULL pairs
+ * every box. fp32 X always takes every box in three parts (X hi/lo x weight
+ * hi/lo, less the lo x lo product). */
+typedef enum { SLIM_SBA_ADAPTIVE = 0, SLIM_SBA_FULL = 1 } slim_sba_precision;
+
 /* Human-readable text of a status code. Never NULL. */
 const char* slim_status_string(int status);
 /* Text of the last CUDA error seen by this thread's calls ("" if none). */
@@ -72,6 +97,13 @@ const char* slim_last_cuda_error(void);
 int slim_last_status_detail(void);
 /* Library version string. */
 const char* slim_version(void);
+
+/* Measured fp64 rates of the current device in TFLOP/s: the fp64 tensor-core
+ * MMA (m8n8k4) and the fp64 FMA pipe, each the best of three short runs of
+ * independent chains on every SM (a few milliseconds in all). Not an operation
+ * of the method: the roofline denominators of its fp64 stages (the inverse
+ * Hessian, the GPTQ update, SQC). Waits for `stream`. */
+int slim_peak_fp64(double* dmma_tflops, double* dfma_tflops, void* stream);
 
 /* Number of SBA candidates, floor(k / 2) + 1 ([P1] 组件一 SBA: the search
  * range of the promoted-group count p is [0, k/2]). */
@@ -152,21 +184,40 @@ int slim_salience_noalloc(const float* W, int64_t m, int64_t n, const double* h,
  * softmax over the m output features, W_p the per-group min-max round-to-
  * nearest dequantization of W under that allocation. p* is the smallest p
  * with the least KL.
- *   order    device k int32 (from slim_salience).
+ *   order    device k int32 (from slim_salience): a permutation of 0..k-1,
+ *            checked on the device (otherwise SLIM_EINVAL).
  *   kl       device P float64 (P = slim_num_candidates), may be NULL.
  *   p_star   device int32, may be NULL.
  *   bits     device k uint8 (the allocation at p*).
  * All candidates are scored in one pass over X: a tensor-core kernel keeps,
  * per token tile, the outputs X W^T and the quantization-error outputs in
  * tensor memory, and updates them group pair by group pair as p grows. The
- * tensor-core operands are fp16 (X converted exactly from bf16; the weight
- * arrays scaled by 2^8): inputs with |x| > 65504 or |w| > 255 return
+ * tensor-core operands are fp16: X converted from bf16 (exact for
+ * |x| >= 2^-17; smaller values round to fp16 subnormals, an absolute error
+ * below 2^-25) or split into two fp16 parts when fp32; each weight-side array
+ * scaled by 2^8, as fp16 values, with the boxes that carry most of the
+ * rounding error held as fp16 hi/lo pairs (22 significant bits; see
+ * slim_sba_precision). Inputs with |x| > 65504 or |w| > 255 return
  * SLIM_ERANGE.
  */
 size_t slim_sba_workspace_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group);
 int slim_sba_search(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N,
                     int group, int avg_bits, const int32_t* order, double* kl, int32_t* p_star,
                     uint8_t* bits, void* ws, size_t ws_bytes, void* stream);
+
+/* slim_sba_search with the scoring objective and the operand precision
+ * selectable: objective is a slim_objective, precision a slim_sba_precision
+ * (slim_sba_search uses SLIM_OBJ_KL, SLIM_SBA_ADAPTIVE). With SLIM_OBJ_MSE, kl receives per candidate the mean over
+ * tokens and outputs of (x W_p^T - x W^T)^2 and p* minimises it. The order
+ * argument is any permutation of the groups: the salience order is the
+ * method; 0, 1, ..., k-1 (promote the first groups, demote the last) is the
+ * head-tail allocation and a random permutation the random allocation of the
+ * method's ablation ([P1] Fig. 5 caption: random / head-tail allocation;
+ * [P2] Measured effects). Workspace: slim_sba_workspace_bytes. */
+int slim_sba_search_ex(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N,
+                       int group, int avg_bits, const int32_t* order, int objective, int precision,
+                       double* kl, int32_t* p_star, uint8_t* bits, void* ws, size_t ws_bytes,
+                       void* stream);
 
 /* ------------------------------------------------------------------------
  * slim_sba_search_split: slim_sba_search's outputs, bit for bit, from a
@@ -212,6 +263,55 @@ int slim_sqc(const float* W, int64_t m, int64_t n, const double* h, const uint8_
              float* zero, uint8_t* tau_idx, void* stream);
 
 /* ------------------------------------------------------------------------
+ * slim_gptq: the quantization of slim_sqc inside the GPTQ layer loop ([P1]
+ * 核心设计: SliM-LLM inserts its two components into GPTQ's layer-wise
+ * quantization skeleton; [P1] FAQ). Columns are taken in order. When the loop
+ * reaches the first column of group c, the group's quantizer is calibrated as
+ * slim_sqc does (bits[c], 3-sigma mask, tau search, element salience w^2/h_j^2
+ * with h = diag(H_d^-1)) on the group's weights as the compensation of the
+ * earlier columns has left them; each column is then rounded with its group's
+ * quantizer, and its error divided by U_jj is subtracted, times row j of U,
+ * from the later columns, where H_d^-1 = U^T U (U upper triangular, H_d = H
+ * with zero diagonal entries set to 1 plus 0.01 mean(diag) on the diagonal).
+ * All arithmetic is fp64; the later columns take each 128-column block's
+ * errors at once (the same sums regrouped).
+ *   H        device n x n float64 (slim_hessian), read only.
+ *   bits     device k uint8 (slim_sba_search), summing to k * avg_bits.
+ *   codes, scale, zero, tau_idx: as slim_sqc (tau_idx may be NULL).
+ * Requires m <= 65535 * 64. Returns SLIM_ENOTPD if H_d has no Cholesky factor.
+ * Workspace: slim_gptq_workspace_bytes (about 8 (2 n^2 + m n) bytes plus the
+ * inverse stage's scratch); ws NULL allocates.
+ */
+size_t slim_gptq_workspace_bytes(int64_t m, int64_t n);
+int slim_gptq(const float* W, int64_t m, int64_t n, const double* H, const uint8_t* bits, int group,
+              int avg_bits, double lambda, int n_tau, uint32_t* codes, float* scale, float* zero,
+              uint8_t* tau_idx, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * slim_dequant_gemv: y = x W_hat^T on the packed layer, the inference product
+ * whose token rate on current GPU kernels the pages name as the method's
+ * limitation for mixed 1/2/3-bit groups ([P1] 局限性; [P2] Limitations).
+ * W_hat[i][j] = scale[i][c] (q_ij - zero[i][c]) with q_ij the code of column j
+ * (group c = j / group) in the layout of slim_sqc.
+ *   codes    device m x slim_row_words(n, avg_bits) uint32 (16-byte aligned).
+ *   bits     device k uint8, each in 1..8, summing to k * avg_bits (the
+ *            caller's precondition: the kernel reads no word outside a row
+ *            whatever bits holds, but y is then unspecified).
+ *   scale, zero  device m x k float32.
+ *   x        device batch x n, row-major, float32 or bf16 (xdtype).
+ *   y        device batch x m float32.
+ * batch is 1..8. Arithmetic: fp32 (each code times x in one fma). The call is
+ * asynchronous: it returns once the kernels are enqueued on `stream` (host-side
+ * argument checks only), so decode loops can issue it back to back. Workspace:
+ * slim_dequant_gemv_workspace_bytes; ws NULL takes it from the library's pool
+ * and returns it in stream order.
+ */
+size_t slim_dequant_gemv_workspace_bytes(int64_t m, int64_t n, int group, int64_t batch);
+int slim_dequant_gemv(const uint32_t* codes, const uint8_t* bits, const float* scale, const float* zero,
+                      int64_t m, int64_t n, int group, int avg_bits, const void* x, int xdtype,
+                      int64_t batch, float* y, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * slim_quantize_layer: the whole path, hessian -> hinv_diag -> salience ->
  * sba_search -> sqc ([P1] 核心设计: SBA allocates bits between groups, SQC
  * calibrates each group's quantizer), with damping alpha = 0.01.
@@ -234,12 +334,35 @@ typedef struct {
   int32_t p_star;     /* HOST, written by the call */
   float stage_ms[8];  /* HOST, written: stages hessian, hinv_diag, salience, sba_search, sqc,
                          total, then the tensor-core kernels alone: hessian (bf16 X), sba scoring */
+  uint8_t* sba_split; /* device (n + 63) / 64 uint8: 1 for the 64-column boxes the SBA scoring
+                         took as fp16 hi/lo pairs (see slim_sba_precision) */
 } slim_diag;
 
 int slim_quantize_layer_ex(const float* W, int64_t m, int64_t n, const void* X, int xdtype,
                            int64_t N, int group, int avg_bits, double lambda, int n_tau,
                            uint32_t* codes, float* scale, float* zero, uint8_t* bits, void* ws,
                            size_t ws_bytes, void* stream, slim_diag* diag);
+
+/* Variants of the whole path, for the method's ablations. A zeroed struct (or
+ * opt == NULL) is the method itself. */
+typedef struct {
+  int objective;         /* slim_objective of the SBA search (default SLIM_OBJ_KL) */
+  int sba_precision;     /* slim_sba_precision of the SBA search (default SLIM_SBA_ADAPTIVE) */
+  int gptq;              /* 0: SQC on the weights as they are (default); 1: the GPTQ column loop
+                            with error compensation (slim_gptq) in place of that SQC stage */
+  const int32_t* order;  /* device k int32, or NULL for the salience order. A caller's
+                            permutation of the groups replaces the salience order in the
+                            search (see slim_sba_search_ex: head-tail, random). Checked on
+                            the device (SLIM_EINVAL if not a permutation). Must not be
+                            diag->order. diag->order then returns this order. */
+} slim_options;
+
+/* slim_quantize_layer_ex with options (opt may be NULL). Workspace:
+ * slim_workspace_bytes. */
+int slim_quantize_layer_opts(const float* W, int64_t m, int64_t n, const void* X, int xdtype,
+                             int64_t N, int group, int avg_bits, double lambda, int n_tau,
+                             uint32_t* codes, float* scale, float* zero, uint8_t* bits, void* ws,
+                             size_t ws_bytes, void* stream, const slim_options* opt, slim_diag* diag);
 
 /* ------------------------------------------------------------------------
  * slim_quantize_layer_host: slim_quantize_layer on HOST arrays (W, X in;

@@ -7,6 +7,7 @@
 #include <cstring>
 #include <string>
 #include <atomic>
+#include <mutex>
 #include <vector>
 
 #include "common.cuh"
@@ -35,18 +36,31 @@ cudaError_t launch_sba_prep_w(const float* W, int64_t m, int64_t n, int64_t N, i
 cudaError_t launch_sba_prep_x(const void* X, int64_t m, int64_t n, int64_t N, int xdtype, int group, int64_t t0,
                               int64_t t1, uint8_t* pw, DevStatus* st, int num_sms, int bps, cudaStream_t s);
 size_t sba_yd_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group);
-cudaError_t launch_sba_phase_a(int64_t m, int64_t n, int xdtype, int64_t N, int group, int tp0, int tp1,
-                               const uint8_t* pw, uint8_t* sw, float* yd, DevStatus* st, int num_sms,
+size_t sba_split_offset(int64_t m, int64_t n, int64_t N, int xdtype, int group, int* nbox);
+cudaError_t launch_sba_phase_a(int64_t m, int64_t n, int xdtype, int64_t N, int group, int objective, int tp0,
+                               int tp1, const uint8_t* pw, uint8_t* sw, float* yd, DevStatus* st, int num_sms,
                                cudaStream_t s);
 cudaError_t launch_sba_steps(int64_t m, int64_t n, int xdtype, int64_t N, int group, int avg_bits,
-                             const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, const uint8_t* pw,
-                             uint8_t* sw, float* yd, DevStatus* st, int num_sms, cudaStream_t s);
+                             const int32_t* order, int objective, double* kl, int32_t* p_star, uint8_t* bits,
+                             const uint8_t* pw, uint8_t* sw, float* yd, DevStatus* st, int num_sms, cudaStream_t s);
 cudaError_t launch_sba_search(int64_t m, int64_t n, int xdtype, int64_t N, int group, int avg_bits,
-                              const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, const uint8_t* pw,
-                              uint8_t* sw, DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev);
+                              const int32_t* order, int objective, double* kl, int32_t* p_star, uint8_t* bits,
+                              const uint8_t* pw, uint8_t* sw, DevStatus* st, int num_sms, cudaStream_t s,
+                              cudaEvent_t* kev);
 cudaError_t launch_sba(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
-                       int avg_bits, const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, uint8_t* ws,
-                       DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev);
+                       int avg_bits, const int32_t* order, int objective, int precision, double* kl, int32_t* p_star,
+                       uint8_t* bits, uint8_t* ws, DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev);
+cudaError_t launch_sba_select(const float* W, const void* X, int64_t m, int64_t n, int64_t N, int xdtype, int group,
+                              int precision, uint8_t* pw, uint8_t* sw, cudaStream_t s);
+cudaError_t launch_order_check(const int32_t* order, int k, int32_t* out, DevStatus* st, cudaStream_t s);
+size_t gptq_workspace_doubles(int64_t m, int64_t n);
+size_t dg_workspace_bytes(int64_t m, int64_t n, int group, int64_t B, int num_sms);
+cudaError_t launch_dequant_gemv(const uint32_t* codes, const uint8_t* bits, const float* scale, const float* zero,
+                                int64_t m, int64_t n, int group, int avg_bits, const void* x, int xdtype, int B,
+                                float* y, uint8_t* ws, int num_sms, cudaStream_t s);
+cudaError_t launch_gptq(const float* W, int64_t m, int64_t n, const double* H, double alpha, const uint8_t* bits,
+                        int group, int avg_bits, double lam, int n_tau, uint32_t* codes, float* scale, float* zero,
+                        uint8_t* tau_idx, double* h, double* ws, DevStatus* st, int num_sms, cudaStream_t s);
 cudaError_t launch_sqc(const float* W, int64_t m, int64_t n, const double* h, const uint8_t* bits, int group,
                        int avg_bits, double lam, int n_tau, uint32_t* codes, float* scale, float* zero,
                        uint8_t* tau_idx, int num_sms, cudaStream_t st);
@@ -119,29 +133,48 @@ int finish(cudaStream_t s, const DevStatus* dst) {
   if (hs.code == kStatusTimeout) return SLIM_ETIMEOUT;
   if (hs.code == kStatusNotPD) return SLIM_ENOTPD;
   if (hs.code == kStatusRangeCode) return SLIM_ERANGE;
+  if (hs.code == kStatusInvalid) return SLIM_EINVAL;
   if (hs.code != 0) return SLIM_ECUDA;
   return SLIM_OK;
 }
 
-// Keep freed stream-ordered allocations in the device's default pool instead of
-// returning them to the driver at every synchronization, so repeated calls
-// that let the library allocate do not re-map gigabytes each time.
-void retain_pool_memory() {
-  thread_local int done_dev = -1;
+constexpr int kMaxDevices = 64;
+
+// The library's own stream-ordered memory pool on the current device (created
+// on first use, kept until the process exits). It keeps freed blocks instead of
+// returning them to the driver at every synchronization, so repeated calls that
+// let the library allocate do not re-map gigabytes each time; being the
+// library's own, it leaves the device's default pool and its settings alone.
+cudaError_t library_pool(cudaMemPool_t* out) {
+  static std::mutex mu;
+  static cudaMemPool_t pools[kMaxDevices] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev == done_dev) return;
-  cudaMemPool_t pool;
-  if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool;
+    e = cudaMemPoolCreate(&pool, &props);
+    if (e != cudaSuccess) return e;
     uint64_t keep = ~0ull;
-    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) { cudaMemPoolDestroy(pool); return e; }
+    pools[dev] = pool;
   }
-  done_dev = dev;
+  *out = pools[dev];
+  return cudaSuccess;
 }
 
 // Workspace holder: caller memory or a cudaMallocAsync'd block freed on scope exit.
 struct Workspace {
   uint8_t* p = nullptr;
   bool owned = false;
+  bool sync_on_release = true;  // false: the stream-ordered free is enough (asynchronous calls)
   cudaStream_t s = nullptr;
   int acquire(void* ws, size_t ws_bytes, size_t need, cudaStream_t st) {
     s = st;
@@ -150,14 +183,18 @@ struct Workspace {
       p = static_cast<uint8_t*>(ws);
       return SLIM_OK;
     }
-    retain_pool_memory();
-    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&p), need, st);
+    cudaMemPool_t pool;
+    cudaError_t e = library_pool(&pool);
+    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&p), need, pool, st);
     if (e != cudaSuccess) { g_last_cuda_error = cudaGetErrorString(e); cudaGetLastError(); return SLIM_ENOMEM; }
     owned = true;
     return SLIM_OK;
   }
   ~Workspace() {
-    if (owned && p) { cudaFreeAsync(p, s); cudaStreamSynchronize(s); }
+    if (owned && p) {
+      cudaFreeAsync(p, s);
+      if (sync_on_release) cudaStreamSynchronize(s);
+    }
   }
 };
 
@@ -177,11 +214,13 @@ struct HostCopy {
   cudaEvent_t pe[2] = {};
   std::vector<cudaEvent_t> ev;
 };
-HostCopy& host_copy(int events) {
-  thread_local HostCopy hc[16];
+// Returns nullptr when the current device cannot be determined or its ordinal
+// is beyond the table.
+HostCopy* host_copy(int events) {
+  thread_local HostCopy hc[kMaxDevices];
   int dev = 0;
-  cudaGetDevice(&dev);
-  HostCopy& x = hc[dev & 15];
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  HostCopy& x = hc[dev];
   if (x.dev != dev) {
     int least = 0, greatest = 0;
     cudaDeviceGetStreamPriorityRange(&least, &greatest);
@@ -199,7 +238,7 @@ HostCopy& host_copy(int events) {
     }
     x.ev.push_back(e);
   }
-  return x;
+  return &x;
 }
 
 // Layout of the full-path workspace. The scratch region holds the SBA
@@ -224,6 +263,7 @@ LayerWs layer_ws(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
   size_t t = sal_bytes(m, n); if (t > rest) rest = t;
   t = sba_search_bytes(m, n, N, xdtype, group); if (t > rest) rest = t;
   t = hessian_ws_bytes(N, n, xdtype); if (t > rest) rest = t;
+  t = gptq_workspace_doubles(m, n) * sizeof(double) + (size_t)n * sizeof(double) + 256; if (t > rest) rest = t;
   const size_t prep = al256(sba_prep_bytes(m, n, N, xdtype, group));
   w.off_scratch = off;
   w.off_rest = off + prep;
@@ -359,14 +399,18 @@ int slim_salience(const float* W, int64_t m, int64_t n, const double* h, int gro
 }
 
 // ------------------------------------------------------------------ sba_search
+// Workspace of the search entries: [status][checked copy of the order][search].
 size_t slim_sba_workspace_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
-  return kStatusBytes + al256(sba_ws_bytes(m, n, N, xdtype, group));
+  if (check_shape(m, n, N, xdtype, group)) return 0;
+  return kStatusBytes + al256((size_t)(n / group) * 4) + al256(sba_ws_bytes(m, n, N, xdtype, group));
 }
 
-int slim_sba_search(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
-                    int avg_bits, const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, void* ws,
-                    size_t ws_bytes, void* stream) {
+int slim_sba_search_ex(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
+                       int avg_bits, const int32_t* order, int objective, int precision, double* kl, int32_t* p_star,
+                       uint8_t* bits, void* ws, size_t ws_bytes, void* stream) {
   if (!W || !X || !order || !bits || !aligned16(W) || !aligned16(X)) return SLIM_EINVAL;
+  if (objective != SLIM_OBJ_KL && objective != SLIM_OBJ_MSE) return SLIM_EINVAL;
+  if (precision != SLIM_SBA_ADAPTIVE && precision != SLIM_SBA_FULL) return SLIM_EINVAL;
   int rc = check_shape(m, n, N, xdtype, group);
   if (rc) return rc;
   rc = check_bits(avg_bits);
@@ -380,14 +424,26 @@ int slim_sba_search(const float* W, int64_t m, int64_t n, const void* X, int xdt
   rc = w.acquire(ws, ws_bytes, slim_sba_workspace_bytes(m, n, N, xdtype, group), s);
   if (rc) return rc;
   DevStatus* st = reinterpret_cast<DevStatus*>(w.p);
+  int32_t* ord = reinterpret_cast<int32_t*>(w.p + kStatusBytes);
+  uint8_t* sw = w.p + kStatusBytes + al256((size_t)(n / group) * 4);
   SLIM_CUDA(cudaMemsetAsync(st, 0, kStatusBytes, s));
-  SLIM_CUDA(launch_sba(W, m, n, X, xdtype, N, group, avg_bits, order, kl, p_star, bits, w.p + kStatusBytes, st,
+  SLIM_CUDA(launch_order_check(order, (int)(n / group), ord, st, s));
+  SLIM_CUDA(launch_sba(W, m, n, X, xdtype, N, group, avg_bits, ord, objective, precision, kl, p_star, bits, sw, st,
                        sms, s, nullptr));
   return finish(s, st);
 }
 
+int slim_sba_search(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
+                    int avg_bits, const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, void* ws,
+                    size_t ws_bytes, void* stream) {
+  return slim_sba_search_ex(W, m, n, X, xdtype, N, group, avg_bits, order, SLIM_OBJ_KL, SLIM_SBA_ADAPTIVE, kl,
+                            p_star, bits, ws, ws_bytes, stream);
+}
+
 size_t slim_sba_split_workspace_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
-  return kStatusBytes + al256(sba_ws_bytes(m, n, N, xdtype, group)) + al256(sba_yd_bytes(m, n, N, xdtype, group));
+  if (check_shape(m, n, N, xdtype, group)) return 0;
+  return kStatusBytes + al256((size_t)(n / group) * 4) + al256(sba_ws_bytes(m, n, N, xdtype, group)) +
+         al256(sba_yd_bytes(m, n, N, xdtype, group));
 }
 
 int slim_sba_search_split(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
@@ -408,19 +464,23 @@ int slim_sba_search_split(const float* W, int64_t m, int64_t n, const void* X, i
   rc = w.acquire(ws, ws_bytes, slim_sba_split_workspace_bytes(m, n, N, xdtype, group), s);
   if (rc) return rc;
   DevStatus* st = reinterpret_cast<DevStatus*>(w.p);
-  uint8_t* pw = w.p + kStatusBytes;
+  int32_t* ord = reinterpret_cast<int32_t*>(w.p + kStatusBytes);
+  uint8_t* pw = w.p + kStatusBytes + al256((size_t)(n / group) * 4);
   const size_t prep = sba_prep_bytes(m, n, N, xdtype, group);
   uint8_t* sw = pw + prep;
   float* yd = reinterpret_cast<float*>(pw + al256(sba_ws_bytes(m, n, N, xdtype, group)));
   SLIM_CUDA(cudaMemsetAsync(st, 0, kStatusBytes, s));
+  SLIM_CUDA(launch_order_check(order, (int)(n / group), ord, st, s));
   SLIM_CUDA(launch_sba_prep_w(W, m, n, N, xdtype, group, avg_bits, pw, st, sms, 8, s));
+  SLIM_CUDA(launch_sba_select(W, X, m, n, N, xdtype, group, SLIM_SBA_ADAPTIVE, pw, sw, s));
   for (int64_t t0 = 0; t0 < N; t0 += chunk_tokens) {
     const int64_t t1 = (t0 + chunk_tokens < N) ? t0 + chunk_tokens : N;
     SLIM_CUDA(launch_sba_prep_x(X, m, n, N, xdtype, group, t0, t1, pw, st, sms, 8, s));
-    SLIM_CUDA(launch_sba_phase_a(m, n, xdtype, N, group, (int)(t0 / 256), (int)((t1 + 255) / 256), pw, sw, yd, st,
-                                 sms, s));
+    SLIM_CUDA(launch_sba_phase_a(m, n, xdtype, N, group, SLIM_OBJ_KL, (int)(t0 / 256), (int)((t1 + 255) / 256), pw,
+                                 sw, yd, st, sms, s));
   }
-  SLIM_CUDA(launch_sba_steps(m, n, xdtype, N, group, avg_bits, order, kl, p_star, bits, pw, sw, yd, st, sms, s));
+  SLIM_CUDA(launch_sba_steps(m, n, xdtype, N, group, avg_bits, ord, SLIM_OBJ_KL, kl, p_star, bits, pw, sw, yd, st,
+                             sms, s));
   return finish(s, st);
 }
 
@@ -445,6 +505,71 @@ int slim_sqc(const float* W, int64_t m, int64_t n, const double* h, const uint8_
   return SLIM_OK;
 }
 
+// ------------------------------------------------------------------ gptq
+size_t slim_gptq_workspace_bytes(int64_t m, int64_t n) {
+  if (m < 1 || n < 1) return 0;
+  return kStatusBytes + al256(gptq_workspace_doubles(m, n) * sizeof(double) + (size_t)n * sizeof(double));
+}
+
+int slim_gptq(const float* W, int64_t m, int64_t n, const double* H, const uint8_t* bits, int group, int avg_bits,
+              double lambda, int n_tau, uint32_t* codes, float* scale, float* zero, uint8_t* tau_idx, void* ws,
+              size_t ws_bytes, void* stream) {
+  if (!W || !H || !bits || !codes || !scale || !zero) return SLIM_EINVAL;
+  int rc = check_shape(m, n, 1, SLIM_X_BF16, group);
+  if (rc) return rc;
+  rc = check_bits(avg_bits);
+  if (rc) return rc;
+  if (!(lambda >= 0.0 && lambda < 1.0) || n_tau < 1 || n_tau > 256) return SLIM_EINVAL;
+  if (m > (int64_t)65535 * 64) return SLIM_EINVAL;
+  int sms = 0;
+  rc = device_sms(&sms);
+  if (rc) return rc;
+  if (injected("gptq")) return SLIM_EINJECTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Workspace w;
+  rc = w.acquire(ws, ws_bytes, slim_gptq_workspace_bytes(m, n), s);
+  if (rc) return rc;
+  DevStatus* st = reinterpret_cast<DevStatus*>(w.p);
+  double* gws = reinterpret_cast<double*>(w.p + kStatusBytes);
+  double* gh = gws + gptq_workspace_doubles(m, n);
+  SLIM_CUDA(cudaMemsetAsync(st, 0, kStatusBytes, s));
+  SLIM_CUDA(launch_gptq(W, m, n, H, kDampAlpha, bits, group, avg_bits, lambda, n_tau, codes, scale, zero, tau_idx, gh,
+                        gws, st, sms, s));
+  return finish(s, st);
+}
+
+// ------------------------------------------------------------------ dequant gemv
+size_t slim_dequant_gemv_workspace_bytes(int64_t m, int64_t n, int group, int64_t batch) {
+  int sms = 0;
+  if (device_sms(&sms) != SLIM_OK) sms = 148;
+  if (m < 1 || n < 1 || group < 32 || n % group || batch < 1) return 0;
+  return al256(dg_workspace_bytes(m, n, group, batch, sms));
+}
+
+int slim_dequant_gemv(const uint32_t* codes, const uint8_t* bits, const float* scale, const float* zero, int64_t m,
+                      int64_t n, int group, int avg_bits, const void* x, int xdtype, int64_t batch, float* y,
+                      void* ws, size_t ws_bytes, void* stream) {
+  if (!codes || !bits || !scale || !zero || !x || !y || !aligned16(codes) || !aligned16(x)) return SLIM_EINVAL;
+  int rc = check_shape(m, n, 1, xdtype, group);
+  if (rc) return rc;
+  rc = check_bits(avg_bits);
+  if (rc) return rc;
+  if (batch < 1 || batch > 8 || (n * avg_bits) % 32) return SLIM_EINVAL;
+  if ((m + 31) / 32 > (int64_t)65535 * 4) return SLIM_EINVAL;
+  int sms = 0;
+  rc = device_sms(&sms);
+  if (rc) return rc;
+  if (injected("dequant_gemv")) return SLIM_EINJECTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Workspace w;
+  w.sync_on_release = false;
+  rc = w.acquire(ws, ws_bytes, slim_dequant_gemv_workspace_bytes(m, n, group, batch), s);
+  if (rc) return rc;
+  SLIM_CUDA(launch_dequant_gemv(codes, bits, scale, zero, m, n, group, avg_bits, x, xdtype, (int)batch, y, w.p, sms,
+                                s));
+  return SLIM_OK;
+}
+
 // ------------------------------------------------------------------ whole layer
 size_t slim_workspace_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group, int avg_bits) {
   (void)avg_bits;
@@ -452,15 +577,24 @@ size_t slim_workspace_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int gro
   return layer_ws(m, n, N, xdtype, group).total;
 }
 
-int slim_quantize_layer_ex(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
-                           int avg_bits, double lambda, int n_tau, uint32_t* codes, float* scale, float* zero,
-                           uint8_t* bits, void* ws, size_t ws_bytes, void* stream, slim_diag* diag) {
+int slim_quantize_layer_opts(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
+                             int avg_bits, double lambda, int n_tau, uint32_t* codes, float* scale, float* zero,
+                             uint8_t* bits, void* ws, size_t ws_bytes, void* stream, const slim_options* opt,
+                             slim_diag* diag) {
   if (!W || !X || !codes || !scale || !zero || !bits || !aligned16(W) || !aligned16(X)) return SLIM_EINVAL;
   int rc = check_shape(m, n, N, xdtype, group);
   if (rc) return rc;
   rc = check_bits(avg_bits);
   if (rc) return rc;
   if (!(lambda >= 0.0 && lambda < 1.0) || n_tau < 1 || n_tau > 256) return SLIM_EINVAL;
+  const int objective = opt ? opt->objective : SLIM_OBJ_KL;
+  const int precision = opt ? opt->sba_precision : SLIM_SBA_ADAPTIVE;
+  const int32_t* given_order = opt ? opt->order : nullptr;
+  if (objective != SLIM_OBJ_KL && objective != SLIM_OBJ_MSE) return SLIM_EINVAL;
+  if (precision != SLIM_SBA_ADAPTIVE && precision != SLIM_SBA_FULL) return SLIM_EINVAL;
+  const bool gptq = opt && opt->gptq != 0;
+  if (opt && opt->gptq != 0 && opt->gptq != 1) return SLIM_EINVAL;
+  if (gptq && m > (int64_t)65535 * 64) return SLIM_EINVAL;
   int sms = 0;
   rc = device_sms(&sms);
   if (rc) return rc;
@@ -479,9 +613,9 @@ int slim_quantize_layer_ex(const float* W, int64_t m, int64_t n, const void* X, 
   uint8_t* tau = diag ? diag->tau_idx : nullptr;
   uint8_t* scratch = w.p + L.off_scratch;
   uint8_t* rest = w.p + L.off_rest;
-  HostCopy& side = host_copy(0);
-  if (!side.ok) return SLIM_ECUDA;
-  JoinOnExit join{s, side.ps, side.pe[1]};
+  HostCopy* side = host_copy(0);
+  if (!side || !side->ok) return SLIM_ECUDA;
+  JoinOnExit join{s, side->ps, side->pe[1]};
 
   cudaEvent_t ev[10] = {};
   const bool timed = diag != nullptr;
@@ -499,20 +633,38 @@ int slim_quantize_layer_ex(const float* W, int64_t m, int64_t n, const void* X, 
     // beside the latency-bound inverse, at most 16K registers per SM (one
     // weight-operand block or two conversion blocks), so that a factorization
     // CTA (about 47K) still fits on every SM
-    SLIM_CUDA(fork_prepare(side, W, m, n, X, xdtype, N, group, avg_bits, scratch, st, sms, 1, 2, s));
+    SLIM_CUDA(fork_prepare(*side, W, m, n, X, xdtype, N, group, avg_bits, scratch, st, sms, 1, 2, s));
     if (injected("hinv_diag")) return SLIM_EINJECTED;
     SLIM_CUDA(launch_hinv(H, n, kDampAlpha, h, reinterpret_cast<double*>(rest), st, s));
     rec(2);
     if (injected("salience")) return SLIM_EINJECTED;
     SLIM_CUDA(launch_salience(W, m, n, h, group, S, order, reinterpret_cast<double*>(rest), s));
+    // a caller's group order replaces the salience order (checked: a
+    // permutation of 0..k-1, else SLIM_EINVAL and the identity is used)
+    if (given_order) SLIM_CUDA(launch_order_check(given_order, (int)(n / group), order, st, s));
     rec(3);
     if (injected("sba_search")) return SLIM_EINJECTED;
-    SLIM_CUDA(join_prepare(side, s));
-    SLIM_CUDA(launch_sba_search(m, n, xdtype, N, group, avg_bits, order, kl, pstar, bits, scratch, rest, st, sms, s,
-                                kev_s));
+    SLIM_CUDA(join_prepare(*side, s));
+    SLIM_CUDA(launch_sba_select(W, X, m, n, N, xdtype, group, precision, scratch, rest, s));
+    SLIM_CUDA(launch_sba_search(m, n, xdtype, N, group, avg_bits, order, objective, kl, pstar, bits, scratch, rest,
+                                st, sms, s, kev_s));
+    if (diag && diag->sba_split) {
+      int nbox = 0;
+      const size_t off = sba_split_offset(m, n, N, xdtype, group, &nbox);
+      SLIM_CUDA(cudaMemcpyAsync(diag->sba_split, scratch + off, (size_t)nbox, cudaMemcpyDeviceToDevice, s));
+    }
     rec(4);
     if (injected("sqc")) return SLIM_EINJECTED;
-    SLIM_CUDA(launch_sqc(W, m, n, h, bits, group, avg_bits, lambda, n_tau, codes, scale, zero, tau, sms, s));
+    if (gptq) {
+      // the GPTQ column loop with SBA's bits and SQC's quantizer, in place of SQC
+      // on the unchanged weights (the diagonal it derives, behind its scratch)
+      double* gws = reinterpret_cast<double*>(rest);
+      double* gh = gws + gptq_workspace_doubles(m, n);
+      SLIM_CUDA(launch_gptq(W, m, n, H, kDampAlpha, bits, group, avg_bits, lambda, n_tau, codes, scale, zero, tau, gh,
+                            gws, st, sms, s));
+    } else {
+      SLIM_CUDA(launch_sqc(W, m, n, h, bits, group, avg_bits, lambda, n_tau, codes, scale, zero, tau, sms, s));
+    }
     rec(5);
     return finish(s, st);
   };
@@ -532,6 +684,13 @@ int slim_quantize_layer_ex(const float* W, int64_t m, int64_t n, const void* X, 
     for (auto& e : ev) cudaEventDestroy(e);
   }
   return rc;
+}
+
+int slim_quantize_layer_ex(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
+                           int avg_bits, double lambda, int n_tau, uint32_t* codes, float* scale, float* zero,
+                           uint8_t* bits, void* ws, size_t ws_bytes, void* stream, slim_diag* diag) {
+  return slim_quantize_layer_opts(W, m, n, X, xdtype, N, group, avg_bits, lambda, n_tau, codes, scale, zero, bits, ws,
+                                  ws_bytes, stream, nullptr, diag);
 }
 
 int slim_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
@@ -611,8 +770,9 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
     const int nsl = (int)((N + stok - 1) / stok);
     const int per = (nsl + 63) / 64;               // slices per chunk: at most 64 chunks
     const int nch = (nsl + per - 1) / per;
-    HostCopy& hc = host_copy(nch + 1);
-    if (!hc.ok) return SLIM_ECUDA;
+    HostCopy* hcp = host_copy(nch + 1);
+    if (!hcp || !hcp->ok) return SLIM_ECUDA;
+    HostCopy& hc = *hcp;
     SLIM_CUDA(cudaMemsetAsync(st, 0, kStatusBytes, s));
     SLIM_CUDA(cudaEventRecord(hc.ev[nch], s));          // the workspace exists before the copies start
     SLIM_CUDA(cudaStreamWaitEvent(hc.cs, hc.ev[nch], 0));
@@ -639,11 +799,14 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
       const int s0 = c * per, cnt = (s0 + per < nsl) ? per : nsl - s0;
       SLIM_CUDA(launch_hessian_slices(dX, N, n, rest, st, sms, s, s0, cnt));
       SLIM_CUDA(cudaStreamWaitEvent(hc.ps, hc.ev[c], 0));
+      // the first chunk holds the token sample of the split selection (a chunk
+      // is at least one 16384-token slice)
+      if (c == 0) SLIM_CUDA(launch_sba_select(dW, dX, m, n, N, xdtype, group, SLIM_SBA_ADAPTIVE, scratch, sw, hc.ps));
       SLIM_CUDA(launch_sba_prep_x(dX, m, n, N, xdtype, group, r0, r1, scratch, st, sms, 2, hc.ps));
       // chunk boundaries are multiples of the slice length, so of 256 tokens:
       // no pair of 128-token tiles straddles two chunks
-      SLIM_CUDA(launch_sba_phase_a(m, n, xdtype, N, group, (int)(r0 / 256), (int)((r1 + 255) / 256), scratch, sw,
-                                   yd, st, sms, hc.ps));
+      SLIM_CUDA(launch_sba_phase_a(m, n, xdtype, N, group, SLIM_OBJ_KL, (int)(r0 / 256), (int)((r1 + 255) / 256),
+                                   scratch, sw, yd, st, sms, hc.ps));
     }
     SLIM_CUDA(launch_hessian_reduce(N, n, rest, H, s));
     if (injected("hinv_diag")) return SLIM_EINJECTED;
@@ -652,8 +815,8 @@ int slim_quantize_layer_host(const float* W, int64_t m, int64_t n, const void* X
     SLIM_CUDA(launch_salience(dW, m, n, h, group, S, order, reinterpret_cast<double*>(rest), s));
     if (injected("sba_search")) return SLIM_EINJECTED;
     SLIM_CUDA(join_prepare(hc, s));
-    SLIM_CUDA(launch_sba_steps(m, n, xdtype, N, group, avg_bits, order, kl, pstar, dbits, scratch, sw, yd, st, sms,
-                               s));
+    SLIM_CUDA(launch_sba_steps(m, n, xdtype, N, group, avg_bits, order, SLIM_OBJ_KL, kl, pstar, dbits, scratch, sw, yd,
+                               st, sms, s));
     if (injected("sqc")) return SLIM_EINJECTED;
     SLIM_CUDA(launch_sqc(dW, m, n, h, dbits, group, avg_bits, lambda, n_tau, dcodes, dscale, dzero, nullptr, sms, s));
     rc = finish(s, st);

@@ -39,6 +39,7 @@ struct DevStatus {
 };
 static_assert(sizeof(DevStatus) == 256, "status area is 256 bytes");
 
+constexpr int kStatusInvalid = 1;   // a device-side argument check failed (SLIM_EINVAL)
 constexpr int kStatusTimeout = 4;
 constexpr int kStatusNotPD = 5;
 constexpr int kStatusRangeCode = 8;
@@ -99,19 +100,30 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // Bounded wait. Returns false (and records SLIM_ETIMEOUT) if the phase did not
 // complete in time or another thread of the CTA already gave up (*abort set).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          DevStatus* st, int where) {
+                                          DevStatus* st, int where, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
+    // the clock is read every 64 polls, or every poll under a shortened limit
+    if ((it & 63u) == 0 || limit_ns != kWaitLimitNs) {
       if (*abort_flag) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         record_failure(st, kStatusTimeout, where);
         return false;
       }
     }
+  }
+}
+
+// Drain wait for work this thread issued itself (its TMA copies, its MMAs):
+// bounded by the same limit but never cut short by an abort, so a CTA that is
+// unwinding still lets its copies land and its MMAs finish before it frees
+// tensor memory and exits.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity) && global_ns() - t0 < kWaitLimitNs) {
   }
 }
 

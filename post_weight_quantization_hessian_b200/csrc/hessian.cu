@@ -106,9 +106,9 @@ __global__ void __launch_bounds__(192, 1) syrk_tc_kernel(const __grid_constant__
           }
         }
       }
-      // let every issued copy land before the CTA can exit
-      for (uint32_t j = (it > HS_STAGES ? it - HS_STAGES : 0); j < it; ++j)
-        mbar_wait(&full[j % HS_STAGES], (j / HS_STAGES) & 1, abort_flag, p.st, 110);
+      // let every issued copy land before the CTA can exit, also after an
+      // abort (bounded, but not cut short by the abort flag)
+      for (uint32_t j = (it > HS_STAGES ? it - HS_STAGES : 0); j < it; ++j) mbar_drain(&full[j % HS_STAGES], (j / HS_STAGES) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -146,8 +146,9 @@ __global__ void __launch_bounds__(192, 1) syrk_tc_kernel(const __grid_constant__
         if (!ok) break;
         tc_commit(tfull);
       }
+      // every issued MMA completes before TMEM can be freed, also after an abort
       tc_commit(done);
-      mbar_wait(done, 0, abort_flag, p.st, 140);
+      mbar_drain(done, 0);
     }
   } else {
     const int wq = warp & 3;

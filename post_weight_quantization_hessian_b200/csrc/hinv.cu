@@ -30,14 +30,11 @@
 #include <cstdint>
 #include <vector>
 #include "common.cuh"
+#include "f64_tiles.cuh"
 
 namespace slim {
 
-constexpr int NB = 64;         // block size
-constexpr int LD = 68;         // shared row stride in doubles: 16-byte rows, conflict-free fragment loads
-constexpr int TILE = NB * LD;  // doubles per shared tile
-constexpr int HT = 256;        // threads per CTA of every blocked kernel
-constexpr size_t kTileBytes = TILE * sizeof(double);
+
 
 __host__ __device__ inline int64_t pad32(int64_t n) { return (n + 31) / 32 * 32; }
 
@@ -65,132 +62,32 @@ __global__ void diag_sum_kernel(const double* __restrict__ H, int64_t n, double 
 }
 
 // A (np x np) = lower triangle of H with the dead-column fix and damping, an
-// identity block on the padding, zeros elsewhere.
+// identity block on the padding, zeros elsewhere. A thread writes two adjacent
+// entries (np is even) with one 16-byte store, grid-stride over the matrix so
+// that a few waves of blocks keep many stores in flight.
 __global__ void damp_copy_kernel(const double* __restrict__ H, int64_t n, int64_t np, const double* __restrict__ damp,
                                  double* __restrict__ A) {
   const double dv = damp[0];
-  for (int64_t i = blockIdx.y; i < np; i += gridDim.y)
-    for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < np; j += (int64_t)gridDim.x * blockDim.x) {
-      double v = 0.0;
+  const int64_t half = np / 2, total = np * half;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = e / half, j0 = 2 * (e - i * half);
+    double v[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int64_t j = j0 + u;
+      double x = 0.0;
       if (i < n && j < n) {
-        if (j < i) v = H[i * n + j];
+        if (j < i) x = H[i * n + j];
         else if (j == i) {
           const double d = H[i * n + i];
-          v = ((d == 0.0) ? 1.0 : d) + dv;
+          x = ((d == 0.0) ? 1.0 : d) + dv;
         }
       } else if (i == j) {
-        v = 1.0;
+        x = 1.0;
       }
-      A[i * np + j] = v;
+      v[u] = x;
     }
-}
-
-// ---------------------------------------------------------------- tiles and fp64 MMA
-__device__ __forceinline__ void cp16(double* sdst, const double* gsrc, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(sdst)), "l"(gsrc),
-               "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
-
-// Queue the copy of a rows x cols block of G (leading dimension ld) into the
-// shared tile S; zeros outside the block. cols is even.
-__device__ __forceinline__ void tile_load_async(double* S, const double* G, int64_t ld, int rows, int cols) {
-#pragma unroll
-  for (int q = 0; q < NB * NB / 2 / HT; ++q) {
-    const int e = threadIdx.x + HT * q;
-    const int r = e >> 5, c = (e & 31) * 2;
-    const bool v = (r < rows) && (c < cols);
-    cp16(S + r * LD + c, v ? G + (int64_t)r * ld + c : G, v);
-  }
-}
-
-// d (8 x 8, two per lane) += a (8 x 4) * b (4 x 8)
-__device__ __forceinline__ void dmma(double (&d)[2], double a, double b) {
-  asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};\n"
-      : "+d"(d[0]), "+d"(d[1])
-      : "d"(a), "d"(b));
-}
-
-// Warp w of 8 owns rows 16 (w >> 1) .. + 15 and columns 32 (w & 1) .. + 31 of a
-// 64 x 64 result: acc[mi][ni] is the 8 x 8 piece at row 16 (w >> 1) + 8 mi,
-// column 32 (w & 1) + 8 ni; a lane holds row (lane >> 2), columns 2 (lane & 3)
-// and 2 (lane & 3) + 1 of each piece.
-using Acc = double[2][4][2];
-
-__device__ __forceinline__ void acc_zero(Acc& acc) {
-#pragma unroll
-  for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-    for (int ni = 0; ni < 4; ++ni) acc[mi][ni][0] = acc[mi][ni][1] = 0.0;
-}
-
-__device__ __forceinline__ int acc_row(int mi) { return 16 * (threadIdx.x >> 6) + 8 * mi + ((threadIdx.x & 31) >> 2); }
-__device__ __forceinline__ int acc_col(int ni) { return 32 * ((threadIdx.x >> 5) & 1) + 8 * ni + 2 * (threadIdx.x & 3); }
-
-__device__ __forceinline__ void acc_from_smem(Acc& acc, const double* S) {
-#pragma unroll
-  for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-    for (int ni = 0; ni < 4; ++ni) {
-      const double2 v = *reinterpret_cast<const double2*>(S + acc_row(mi) * LD + acc_col(ni));
-      acc[mi][ni][0] = v.x;
-      acc[mi][ni][1] = v.y;
-    }
-}
-__device__ __forceinline__ void acc_to_smem(const Acc& acc, double* S) {
-#pragma unroll
-  for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-    for (int ni = 0; ni < 4; ++ni)
-      *reinterpret_cast<double2*>(S + acc_row(mi) * LD + acc_col(ni)) = make_double2(acc[mi][ni][0], acc[mi][ni][1]);
-}
-__device__ __forceinline__ void acc_from_global(Acc& acc, const double* G, int64_t ld, int rows, int cols) {
-#pragma unroll
-  for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-    for (int ni = 0; ni < 4; ++ni) {
-      const int r = acc_row(mi), c = acc_col(ni);
-      double2 v = make_double2(0.0, 0.0);
-      if (r < rows && c < cols) v = *reinterpret_cast<const double2*>(G + (int64_t)r * ld + c);
-      acc[mi][ni][0] = v.x;
-      acc[mi][ni][1] = v.y;
-    }
-}
-__device__ __forceinline__ void acc_to_global(const Acc& acc, double* G, int64_t ld, int rows, int cols) {
-#pragma unroll
-  for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-    for (int ni = 0; ni < 4; ++ni) {
-      const int r = acc_row(mi), c = acc_col(ni);
-      if (r < rows && c < cols)
-        *reinterpret_cast<double2*>(G + (int64_t)r * ld + c) = make_double2(acc[mi][ni][0], acc[mi][ni][1]);
-    }
-}
-
-// acc += (NEG ? -1 : 1) * sum_{k < kn} As[row][k] * B(k, col), kn a multiple of 4.
-// BT: Bs holds B transposed (Bs[col][k], the product is As Bs^T); else Bs[k][col].
-template <bool BT, bool NEG>
-__device__ __forceinline__ void warp_mma64(Acc& acc, const double* As, const double* Bs, int kn) {
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, kq = lane & 3;
-  const double* a0 = As + (16 * (w >> 1) + g) * LD + kq;
-  const int cb = 32 * (w & 1) + g;
-#pragma unroll 4
-  for (int k = 0; k < kn; k += 4) {
-    double a[2], b[4];
-    a[0] = a0[k];
-    a[1] = a0[8 * LD + k];
-    if (NEG) {
-      a[0] = -a[0];
-      a[1] = -a[1];
-    }
-#pragma unroll
-    for (int ni = 0; ni < 4; ++ni) b[ni] = BT ? Bs[(cb + 8 * ni) * LD + k + kq] : Bs[(k + kq) * LD + cb + 8 * ni];
-#pragma unroll
-    for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-      for (int ni = 0; ni < 4; ++ni) dmma(acc[mi][ni], a[mi], b[ni]);
+    *reinterpret_cast<double2*>(A + i * np + j0) = make_double2(v[0], v[1]);
   }
 }
 
@@ -606,20 +503,31 @@ __global__ void __launch_bounds__(HT, 3) inv_update_kernel(const double* __restr
 }
 
 // ---------------------------------------------------------------- column norms
-constexpr int kNormRows = 128;
+constexpr int kNormRows = 64;
+constexpr int kSmsHint = 148;  // grid size hint of the streaming copy (a few blocks per SM)
+// Partial column sums of squares of the lower triangle of M over runs of
+// kNormRows rows; four independent chains per thread keep four loads in flight.
 __global__ void colsumsq_partial_kernel(const double* __restrict__ M, int64_t ld, int64_t n,
                                         double* __restrict__ part) {
   const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= n) return;
-  int64_t i0 = (int64_t)blockIdx.y * kNormRows;
-  int64_t i1 = i0 + kNormRows < ld ? i0 + kNormRows : ld;
-  if (i0 < j) i0 = j;
-  double acc = 0.0;
-  for (int64_t i = i0; i < i1; ++i) {
-    const double v = M[i * ld + j];
-    acc = fma(v, v, acc);
+  const int64_t r0 = (int64_t)blockIdx.y * kNormRows;
+  const int64_t i1 = r0 + kNormRows < ld ? r0 + kNormRows : ld;
+  const int64_t i0 = r0 < j ? j : r0;
+  double a[4] = {0.0, 0.0, 0.0, 0.0};
+  int64_t i = i0;
+  for (; i + 3 < i1; i += 4) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const double v = M[(i + u) * ld + j];
+      a[u] = fma(v, v, a[u]);
+    }
   }
-  part[(int64_t)blockIdx.y * n + j] = acc;
+  for (; i < i1; ++i) {
+    const double v = M[i * ld + j];
+    a[0] = fma(v, v, a[0]);
+  }
+  part[(int64_t)blockIdx.y * n + j] = (a[0] + a[1]) + (a[2] + a[3]);
 }
 __global__ void colsumsq_final_kernel(const double* __restrict__ part, int nparts, int64_t n, double* __restrict__ h) {
   const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -682,8 +590,7 @@ static int enqueue_hinv(const double* H, int64_t n, double alpha, double* h, dou
   double* damp = part + parts * n;
   const int T = (int)((np + NB - 1) / NB);
   diag_sum_kernel<<<1, 1024, 0, o>>>(H, n, alpha, damp);
-  damp_copy_kernel<<<dim3((unsigned)((np + 255) / 256), (unsigned)(np < 65535 ? np : 65535)), 256, 0, o>>>(H, n, np, damp,
-                                                                                                      A);
+  damp_copy_kernel<<<kSmsHint * 8, 256, 0, o>>>(H, n, np, damp, A);
   cudaMemsetAsync(M, 0, (size_t)np * np * sizeof(double), o);
   cudaEvent_t* ePP = hs.ev.data();
   cudaEvent_t* eTr = ePP + T;

@@ -91,6 +91,34 @@ cudaError_t launch_salience(const float* W, int64_t m, int64_t n, const double* 
   return cudaGetLastError();
 }
 
+// A caller's order of the k groups (device), checked to be a permutation of
+// 0..k-1 and copied to `out`; if it is not, the identity is written instead
+// (so later kernels never index outside the groups) and SLIM_EINVAL recorded.
+// One block of 1024 threads; k <= 1024.
+__global__ void order_check_kernel(const int32_t* __restrict__ order, int k, int32_t* __restrict__ out,
+                                   DevStatus* st) {
+  __shared__ int seen[1024];
+  __shared__ int bad;
+  for (int c = threadIdx.x; c < k; c += blockDim.x) seen[c] = 0;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  for (int c = threadIdx.x; c < k; c += blockDim.x) {
+    const int v = order[c];
+    if (v < 0 || v >= k || atomicAdd(&seen[v], 1) != 0) atomicExch(&bad, 1);
+  }
+  __syncthreads();
+  const bool ok = bad == 0;
+  for (int c = threadIdx.x; c < k; c += blockDim.x) out[c] = ok ? order[c] : c;
+  if (!ok && threadIdx.x == 0) record_failure(st, kStatusInvalid, 0);
+}
+
+cudaError_t launch_order_check(const int32_t* order, int k, int32_t* out, DevStatus* st, cudaStream_t s) {
+  if (k < 1 || k > 1024) return cudaErrorInvalidValue;
+  order_check_kernel<<<1, 1024, 0, s>>>(order, k, out, st);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 }  // namespace slim
 
 namespace slim {

@@ -20,12 +20,22 @@
 // full K = n contraction, then add the two changed groups' K = 2g slices for
 // every further p. After each step the epilogue reads d_p from TMEM and
 // accumulates the softmax statistics. d carries the quantization error
-// directly (not as a difference of two large products). Operands are fp16
-// (11-bit significand): X converted from bf16 exactly, the weight-side arrays
-// scaled by 2^8 (exact) so small entries stay out of fp16 subnormals, and the
-// fp32 accumulators scaled back by 2^-8. Tensor-core work: 2Nnm (y) + 2Nnm
-// (d_0) + (P-1) 4Ngm (updates), instead of P 2Nnm for one dequant-GEMM per
-// candidate.
+// directly (not as a difference of two large products).
+//
+// Operands. X is fp16: converted exactly from bf16, or split into a high and a
+// low fp16 part when it is fp32. Each weight-side array (W, E0, Dp, Dm) is
+// scaled by 2^8 (exact; keeps small entries out of fp16 subnormals) and stored
+// as an fp16 pair, v 2^8 = hi + lo with hi = RN16(v 2^8), lo = RN16(v 2^8 - hi):
+// 22 significant bits instead of fp16's 11. A single fp16 copy of the weight
+// side moves the output KL by up to several 1e-5 on layers with clustered
+// activation outliers (its rounding error in y = X W^T is largest exactly
+// where the outlier channels meet the salient weights); the pair removes that
+// term. Every K box is therefore contracted as sub-chunks that share the X
+// box: (X, hi) and (X, lo) for bf16 X; (X_hi, hi), (X_lo, hi), (X_hi, lo) for
+// fp32 X (X_lo lo, about 2^-22 of the product, is left out). The fp32
+// accumulators are scaled back by 2^-8. Executed tensor-core work:
+// nsub (2Nnm (y) + 2Nnm (d_0) + (P-1) 4Ngm (updates)), nsub = 2 or 3, instead
+// of P 2Nnm for one dequant-GEMM per candidate.
 //
 // KL from running sums, per token t and output range (with e_y = exp(y - M)):
 //   S_y = sum e_y, S_q = sum e_y exp(d), A = sum e_y d
@@ -35,7 +45,8 @@
 //
 // Kernels
 //   sba_prep       warp per (row, group): RTN at b-1, b, b+1 in fp64 (the
-//                  definition's operation order); writes fp16 2^8 W, E0, Dp, Dm
+//                  definition's operation order); writes the fp16 hi/lo pairs
+//                  of 2^8 W, E0, Dp, Dm
 //   x_to_f16       bf16 X -> fp16 (exact in fp16's normal range)
 //   x_split        fp32 X: X ~ X_hi + X_lo as two fp16 halves of X_cat
 //   sba_score      persistent tcgen05 kernel (below)
@@ -43,6 +54,7 @@
 //                  sums per token tile
 //   sba_final      KL_p = sum / N, p* = first argmin, bits
 #include <cstdint>
+#include <cstdlib>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include "common.cuh"
@@ -61,13 +73,24 @@ __device__ __forceinline__ __half to_half_checked(float v, DevStatus* st, int wh
   return __float2half_rn(v);
 }
 
+// v = hi + lo as two fp16 values (hi = RN16(v), lo = RN16(v - hi); v - hi is
+// exact in fp64), hi range-checked.
+__device__ __forceinline__ void split_half(double v, DevStatus* st, int where, __half& hi, __half& lo) {
+  if (!(fabs(v) <= (double)kHalfMax)) record_failure(st, kStatusRange, where);
+  hi = __double2half(v);
+  lo = __double2half(v - (double)__half2float(hi));
+}
+
 // Weight-side operands. W is read as float4: a lane holds 4 consecutive
 // weights, a group of G spans G/4 adjacent lanes (G divides 128 and n, so a
-// group never leaves its lanes or its row), and each output array gets one
-// 8-byte store per lane. Per group: fp32 min/max, then per level b-1, b, b+1
-// the fp64 min-max RTN value.
+// group never leaves its lanes or its row). Per group: fp32 min/max, then per
+// level b-1, b, b+1 the fp64 min-max RTN value. Each output array is row-major
+// with rows of 2 npad fp16 values: the hi parts in columns [0, npad), the lo
+// parts in [npad, 2 npad); a lane writes one 8-byte word to each half
+// (rs2 = 2 npad / 4 and lo2 = npad / 4 in those words).
 template <int G>
-__global__ void __launch_bounds__(256) sba_prep_kernel(const float4* __restrict__ W, int64_t total4, int avg_bits,
+__global__ void __launch_bounds__(256) sba_prep_kernel(const float4* __restrict__ W, int64_t total4, int64_t n4,
+                                                       int64_t rs2, int64_t lo2, int avg_bits,
                                                        uint2* __restrict__ Wb, uint2* __restrict__ E0,
                                                        uint2* __restrict__ Dp, uint2* __restrict__ Dm,
                                                        DevStatus* st) {
@@ -110,19 +133,25 @@ __global__ void __launch_bounds__(256) sba_prep_kernel(const float4* __restrict_
         wh[l][r] = deg ? wd : s0 * (q - z0);
       }
     }
-    __half o0[4], o1[4], o2[4], o3[4];
+    __half h0[4], h1[4], h2[4], h3[4], l0[4], l1[4], l2[4], l3[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const double wd = w[r];
-      o0[r] = to_half_checked(w[r] * kOpScale, st, 300);
-      o1[r] = to_half_checked((float)(wh[1][r] - wd) * kOpScale, st, 301);
-      o2[r] = to_half_checked((float)(wh[2][r] - wh[1][r]) * kOpScale, st, 302);
-      o3[r] = to_half_checked((float)(wh[0][r] - wh[1][r]) * kOpScale, st, 303);
+      split_half(wd * (double)kOpScale, st, 300, h0[r], l0[r]);
+      split_half((wh[1][r] - wd) * (double)kOpScale, st, 301, h1[r], l1[r]);
+      split_half((wh[2][r] - wh[1][r]) * (double)kOpScale, st, 302, h2[r], l2[r]);
+      split_half((wh[0][r] - wh[1][r]) * (double)kOpScale, st, 303, h3[r], l3[r]);
     }
-    Wb[e] = *reinterpret_cast<const uint2*>(o0);
-    E0[e] = *reinterpret_cast<const uint2*>(o1);
-    Dp[e] = *reinterpret_cast<const uint2*>(o2);
-    Dm[e] = *reinterpret_cast<const uint2*>(o3);
+    const int64_t row = e / n4;
+    const int64_t o = row * rs2 + (e - row * n4);
+    Wb[o] = *reinterpret_cast<const uint2*>(h0);
+    E0[o] = *reinterpret_cast<const uint2*>(h1);
+    Dp[o] = *reinterpret_cast<const uint2*>(h2);
+    Dm[o] = *reinterpret_cast<const uint2*>(h3);
+    Wb[o + lo2] = *reinterpret_cast<const uint2*>(l0);
+    E0[o + lo2] = *reinterpret_cast<const uint2*>(l1);
+    Dp[o + lo2] = *reinterpret_cast<const uint2*>(l2);
+    Dm[o + lo2] = *reinterpret_cast<const uint2*>(l3);
   }
 }
 
@@ -189,14 +218,17 @@ struct SbaTmaps {
 
 struct SbaParams {
   int64_t N, m, n;
-  int g, k, P, ksplit;
+  int npad;                      // weight-side row half: n rounded up to whole 64-column boxes
+  int g, k, P, ksplit, nsub;     // nsub: 3 for fp32 X (every box); 2 for bf16 X (split boxes only)
+  int nbox;                      // 64-wide K boxes, (n + 63) / 64
+  const uint8_t* split;          // [nbox] 1: the box's weight side is taken as hi and lo (bf16 X)
   int n_tt, n_tp, n_ot, stages;  // token tiles, token-tile pairs, output tiles
-  int nA, nD;                    // chunks of phase A and of one delta step
   const int32_t* order;
   float* part;                   // [n_tt][n_ot][F][128], F = 2 + 2P
   float* yd;                     // split runs: [n_tt][n_ot][e^(y-M), d][128 outputs][128 tokens]
   int tp0;                       // first token-tile pair of this launch (n_tp pairs from there)
   DevStatus* st;
+  uint64_t acc_wait_ns;          // limit of the epilogue's wait for an accumulator (normally kWaitLimitNs)
 };
 
 struct Chunk {
@@ -204,46 +236,73 @@ struct Chunk {
   int which;  // 0: phase A (Wb, E0); 1: Dp; 2: Dm
 };
 
-// Per-item chunk geometry without divisions in the chunk loop. Step 0 is phase
-// A (y = X Wb^T, d = X E0^T over K = n; chunk c is K box c >> (ksplit - 1),
-// X half c & (ksplit - 1)); step p >= 1 adds the promoted group order[p-1]
-// (Dp) and the demoted group order[k-p] (Dm), promoted chunks first.
+// Sub-chunks. Every 64-wide K box is contracted as 1, 2 or 3 consecutive
+// sub-chunks that share the box's X and weight columns:
+//   bf16 X, box not split: (X, hi)
+//   bf16 X, box split:     (X, hi), (X, lo)
+//   fp32 X (every box):    (X_hi, hi), (X_lo, hi), (X_hi, lo)
+// X_lo sits n columns after X_hi, a weight lo part npad columns after its hi
+// part. s_split[b] (shared memory) marks the split boxes; sub_count(b) is the
+// number of sub-chunks of box b.
+__device__ __forceinline__ int sub_count(const SbaParams& p, const uint8_t* s_split, int b) {
+  return p.nsub == 3 ? 3 : 1 + s_split[b];
+}
+
+// Per-item chunk geometry. Step 0 is phase A (y = X Wb^T, d = X E0^T over
+// K = n), its chunks listed in s_tab (box << 2 | sub). Step p >= 1 adds the
+// promoted group order[p-1] (Dp) and the demoted group order[k-p] (Dm),
+// promoted chunks first; a group covers one box (g <= 64) or two (g = 128).
 struct ItemGeom {
-  int step, ks_shift, per_group, col_up, col_dn, k16_lo_up, k16_lo_dn, k16_n;
+  int step, nch, n_up, box_up, box_dn, k16_lo_up, k16_lo_dn, k16_n, up0, dn0;  // up0/dn0: sub-chunks of a group's first box
 };
-__device__ __forceinline__ ItemGeom item_geom(const SbaParams& p, const int32_t* order, int step) {
+__device__ __forceinline__ ItemGeom item_geom(const SbaParams& p, const int32_t* order, const uint8_t* s_split,
+                                              int nA, int step) {
   ItemGeom g;
   g.step = step;
-  g.ks_shift = p.ksplit == 2 ? 1 : 0;
-  g.per_group = p.nD >> 1;
   g.k16_n = p.g >= 64 ? 4 : p.g / 16;
-  g.col_up = g.col_dn = 0;
+  g.box_up = g.box_dn = 0;
   g.k16_lo_up = g.k16_lo_dn = 0;
-  if (step > 0) {
-    const int cu = order[step - 1] * p.g, cd = order[p.k - step] * p.g;
-    g.col_up = p.g >= 64 ? cu : (cu & ~63);
-    g.col_dn = p.g >= 64 ? cd : (cd & ~63);
-    g.k16_lo_up = p.g >= 64 ? 0 : (cu & 63) >> 4;
-    g.k16_lo_dn = p.g >= 64 ? 0 : (cd & 63) >> 4;
+  g.up0 = g.dn0 = 0;
+  if (step == 0) {
+    g.nch = nA;
+    g.n_up = nA;
+    return g;
   }
+  const int cu = order[step - 1] * p.g, cd = order[p.k - step] * p.g;
+  g.box_up = cu >> 6;
+  g.box_dn = cd >> 6;
+  g.k16_lo_up = p.g >= 64 ? 0 : (cu & 63) >> 4;
+  g.k16_lo_dn = p.g >= 64 ? 0 : (cd & 63) >> 4;
+  g.up0 = sub_count(p, s_split, g.box_up);
+  g.dn0 = sub_count(p, s_split, g.box_dn);
+  g.n_up = g.up0 + (p.g == 128 ? sub_count(p, s_split, g.box_up + 1) : 0);
+  g.nch = g.n_up + g.dn0 + (p.g == 128 ? sub_count(p, s_split, g.box_dn + 1) : 0);
   return g;
 }
-__device__ __forceinline__ void chunk_at(const SbaParams& p, const ItemGeom& g, int c, Chunk& ch) {
-  const int sx = c & ((1 << g.ks_shift) - 1);
+__device__ __forceinline__ void chunk_at(const SbaParams& p, const ItemGeom& g, const uint16_t* s_tab, int c,
+                                         Chunk& ch) {
+  int box, sub;
   if (g.step == 0) {
-    ch.bcol = (c >> g.ks_shift) * SB_BK;
+    box = s_tab[c] >> 2;
+    sub = s_tab[c] & 3;
     ch.k16_lo = 0;
     ch.k16_hi = 4;
     ch.which = 0;
   } else {
-    const bool up = c < g.per_group;
-    const int rem = up ? c : c - g.per_group;
-    ch.bcol = (up ? g.col_up : g.col_dn) + (rem >> g.ks_shift) * SB_BK;
+    const bool up = c < g.n_up;
+    const int l = up ? c : c - g.n_up;
+    const int first = up ? g.up0 : g.dn0;
+    box = (up ? g.box_up : g.box_dn) + (l >= first ? 1 : 0);
+    sub = l >= first ? l - first : l;
     ch.k16_lo = up ? g.k16_lo_up : g.k16_lo_dn;
     ch.k16_hi = ch.k16_lo + g.k16_n;
     ch.which = up ? 1 : 2;
   }
-  ch.xcol = ch.bcol + (sx ? (int)p.n : 0);
+  const int xs = (p.nsub == 3 && sub == 1) ? 1 : 0;      // X_lo
+  const int bs = (sub == (p.nsub == 3 ? 2 : 1)) ? 1 : 0;  // weight lo part
+  const int col = box * SB_BK;
+  ch.xcol = col + (xs ? (int)p.n : 0);
+  ch.bcol = col + (bs ? p.npad : 0);
 }
 
 // Work unit u -> (token-tile pair, output tile); raster bands of SB_BAND pairs.
@@ -268,6 +327,11 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^k for an integral k <= 0 (exact; 0 below the normal range).
+__device__ __forceinline__ float pow2i(float k) {
+  return k >= -126.f ? __int_as_float((127 + (int)k) << 23) : 0.f;
+}
+
 // Packed fp32 pairs (sm_100 f32x2 arithmetic): the epilogue handles two output
 // columns per instruction, which leaves more issue slots to the MMA thread on
 // the same SM sub-partition.
@@ -290,6 +354,13 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   return d;
 }
 
+// max(a, b, c) in one instruction (sm_100 three-input max).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // One work unit is two token tiles (TMEM slots 0 and 1) against one output tile:
 // every weight-side box feeds both slots' MMAs, so per output tile the kernel
 // moves about a third fewer bytes than with one token tile.
@@ -307,7 +378,7 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
 // stores each tile's e^(y - M) and d, exactly as they sit in TMEM after phase
 // A; kSbaSteps loads them back into TMEM and continues with step 1, so the
 // two launches together compute bit for bit what one kSbaAll launch does.
-template <int MODE>
+template <int MODE, int OBJ>
 __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_constant__ SbaTmaps tm, SbaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -321,14 +392,23 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
   uint32_t* tslot = reinterpret_cast<uint32_t*>(xbar + 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   int32_t* s_order = reinterpret_cast<int32_t*>(tslot + 2);
-  float* s_x = reinterpret_cast<float*>(s_order + ((p.k + 3) & ~3));  // [2 slots][128 rows][8]
+  float* s_x = reinterpret_cast<float*>(s_order + ((p.k + 3) & ~3));  // [2 slots][128 rows][12]
+  uint16_t* s_tab = reinterpret_cast<uint16_t*>(s_x + 2 * 128 * 12);    // phase-A chunks: box << 2 | sub
+  uint8_t* s_split = reinterpret_cast<uint8_t*>(s_tab + 3 * p.nbox);   // [nbox]
+  int* s_na = reinterpret_cast<int*>(s_split + ((p.nbox + 15) & ~15));  // chunks of phase A
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int s_lo = MODE == kSbaSteps ? 1 : 0;  // the launch's steps: [s_lo, s_hi)
   const int s_hi = MODE == kSbaPhaseA ? 1 : p.P;
   if (MODE != kSbaPhaseA)
     for (int c = threadIdx.x; c < p.k; c += blockDim.x) s_order[c] = p.order[c];
+  for (int b = threadIdx.x; b < p.nbox; b += blockDim.x) s_split[b] = p.nsub == 3 ? 0 : (p.split[b] ? 1 : 0);
+  __syncthreads();
   if (threadIdx.x == 0) {
+    int c = 0;
+    for (int b = 0; b < p.nbox; ++b)
+      for (int u = 0; u < sub_count(p, s_split, b); ++u) s_tab[c++] = (uint16_t)(b << 2 | u);
+    *s_na = c;
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int s = 0; s < 2; ++s) { mbar_init(&afull[s], 1); mbar_init(&afree[s], SB_EPI_WARPS / 2); }
     mbar_init(done, 1);
@@ -341,6 +421,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tbase = *tslot;
   const int units = p.n_tp * p.n_ot;
+  const int nA = *s_na;
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
@@ -354,11 +435,11 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
         unit_decode(p, u, tp, ot);
         const int xrow0 = 2 * tp * SB_BM, xrow1 = xrow0 + SB_BM, brow = ot * SB_BN;
         for (int step = s_lo; step < s_hi && ok; ++step) {
-          const ItemGeom geo = item_geom(p, s_order, step);
-          const int nch = step == 0 ? p.nA : p.nD;
+          const ItemGeom geo = item_geom(p, s_order, s_split, nA, step);
+          const int nch = geo.nch;
           for (int c = 0; c < nch; ++c) {
             Chunk ch;
-            chunk_at(p, geo, c, ch);
+            chunk_at(p, geo, s_tab, c, ch);
             if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, p.st, 200 + st)) { ok = false; break; }
             uint8_t* sb = smem + st * SB_STAGE;
             mbar_arrive_expect_tx(&full[st], (ch.which == 0 ? 4 : 3) * SB_BOX);
@@ -377,10 +458,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
         }
       }
       // let every issued copy land before the CTA can exit
-      for (uint32_t j = (it > (uint32_t)S ? it - S : 0); j < it; ++j) {
-        uint64_t t0 = global_ns();
-        while (!mbar_try_wait(&full[j % S], (j / S) & 1) && global_ns() - t0 < kWaitLimitNs) {}
-      }
+      for (uint32_t j = (it > (uint32_t)S ? it - S : 0); j < it; ++j) mbar_drain(&full[j % S], (j / S) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
@@ -409,9 +487,8 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           if (!mbar_wait(&afree[0], (cnt & 1) ^ fpar, abort_flag, p.st, 220) ||
               !mbar_wait(&afree[1], (cnt & 1) ^ fpar, abort_flag, p.st, 221)) { ok = false; break; }
           tc_fence_after();
-          ItemGeom geo;
-          if (step > 0 && !dfull) geo = item_geom(p, s_order, step);
-          const int nch = step == 0 ? p.nA : p.nD;
+          const ItemGeom geo = item_geom(p, s_order, s_split, nA, step);
+          const int nch = geo.nch;
           // A shared-memory access by this thread while its MMAs are in flight
           // waits for them to drain (about 380 cycles: the queue holds only a few
           // MMAs), so each wait is made to cover two chunks where it can: right
@@ -445,7 +522,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
                 }
               } else {
                 Chunk ch;
-                chunk_at(p, geo, c, ch);
+                chunk_at(p, geo, s_tab, c, ch);
                 for (int k16 = ch.k16_lo; k16 < ch.k16_hi; ++k16) {
                   tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, 1u);
                   tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, 1u);
@@ -462,8 +539,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
         }
       }
       tc_commit(done);
-      uint64_t t0 = global_ns();
-      while (!mbar_try_wait(done, 0) && global_ns() - t0 < kWaitLimitNs) {}
+      mbar_drain(done, 0);
     }
   } else {
     // ------------------------------------------------ epilogue
@@ -474,7 +550,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
     const int r = q * 32 + lane;
     const int F = 2 + 2 * p.P;
     const uint32_t ty = tbase + ((uint32_t)(q * 32) << 16) + slot * 256 + h * 64, td = ty + 128;
-    float* xs = s_x + (slot * 128 + r) * 8;   // [0..3] even steps, [4..7] odd steps
+    float* xs = s_x + (slot * 128 + r) * 12;  // [0..3] even steps, [4..7] odd steps, [8..9] shifts
     uint64_t* xb = xbar + (slot * 4 + q) * 4;  // max h0, max h1, sums (even), sums (odd)
     uint32_t cnt = 0, nunit = 0;
     bool ok = true;
@@ -508,7 +584,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
         if (lane == 0) mbar_arrive(&afree[slot]);
       }
       for (int step = s_lo; step < s_hi; ++step) {
-        if (!mbar_wait(&afull[slot], cnt & 1, abort_flag, p.st, 240 + slot)) { ok = false; break; }
+        if (!mbar_wait(&afull[slot], cnt & 1, abort_flag, p.st, 240 + slot, p.acc_wait_ns)) { ok = false; break; }
         tc_fence_after();
         uint32_t v[64];
         float sy = 0.f;
@@ -557,37 +633,59 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           __syncwarp();
           if (lane == 0) mbar_arrive(&afree[slot]);
         }
+        // Per-token sums over this thread's 64 outputs. KL: S_q = sum e^(y-M) e^d
+        // and A = sum e^(y-M) d. MSE: the sum of d^2 (accumulator units, x 2^16).
         uint64_t sqp = 0, ap = 0;  // packed (even, odd column) sums
-        const uint64_t kc2 = f2_pack(kC1, kC1);
-        // e^(y - M) in 8-column pieces. In the split launches the pieces are
-        // double-buffered (the load of the next one is in flight while this one
-        // is consumed); the one-pass launch, whose step-0 code already holds
-        // more registers, loads them one at a time. Same arithmetic either way.
-        constexpr int NB = MODE == kSbaAll ? 1 : 2;
-        uint32_t ev[NB][8];
-        if (NB == 2) {
-          tmem_ld8(ty, ev[0]);
-          tc_wait_ld8(ev[0]);
-        }
+        float csh = 0.f;           // S_q carries a factor 2^-csh (0 unless it could overflow)
+        if (OBJ == 1) {
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          uint32_t (&cur)[8] = ev[cc % NB];
-          if (NB == 1) {
-            tmem_ld8(ty + cc * 8, cur);
-            tc_wait_ld8(cur);
-          } else if (cc + 1 < 8) {
-            tmem_ld8(ty + (cc + 1) * 8, ev[(cc + 1) % NB]);
+          for (int j = 0; j < 64; j += 2) {
+            const uint64_t dd = f2_pack(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+            sqp = f2_fma(dd, dd, sqp);
+          }
+        } else {
+          // A quantized output far above its full-precision value (d above about
+          // 44 in output units) would overflow e^d in fp32. The thread's largest
+          // exponent decides a shift csh, a multiple of 32 that keeps every term
+          // at most 2^64; it is 0 for ordinary layers, where e^(d log2(e) - 0)
+          // is exactly the unshifted term.
+          float dm = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+#pragma unroll
+          for (int j = 3; j < 63; j += 2) dm = fmax3(dm, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+          dm = fmaxf(dm, __uint_as_float(v[63]));
+          const float c = dm * kC1 - 64.f;
+          csh = c > 0.f ? 32.f * ceilf(c * (1.f / 32.f)) : 0.f;
+          const uint64_t kc2 = f2_pack(kC1, kC1), nc = f2_pack(-csh, -csh);
+          // e^(y - M) in 8-column pieces. In the split launches the pieces are
+          // double-buffered (the load of the next one is in flight while this one
+          // is consumed); the one-pass launch, whose step-0 code already holds
+          // more registers, loads them one at a time. Same arithmetic either way.
+          constexpr int NB = MODE == kSbaAll ? 1 : 2;
+          uint32_t ev[NB][8];
+          if (NB == 2) {
+            tmem_ld8(ty, ev[0]);
+            tc_wait_ld8(ev[0]);
           }
 #pragma unroll
-          for (int j = 0; j < 8; j += 2) {
-            const uint64_t ey = f2_pack(__uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
-            const uint64_t dd = f2_pack(__uint_as_float(v[cc * 8 + j]), __uint_as_float(v[cc * 8 + j + 1]));
-            float x0, x1;
-            f2_unpack(f2_mul(dd, kc2), x0, x1);
-            sqp = f2_fma(ey, f2_pack(ex2(x0), ex2(x1)), sqp);
-            ap = f2_fma(ey, dd, ap);
+          for (int cc = 0; cc < 8; ++cc) {
+            uint32_t (&cur)[8] = ev[cc % NB];
+            if (NB == 1) {
+              tmem_ld8(ty + cc * 8, cur);
+              tc_wait_ld8(cur);
+            } else if (cc + 1 < 8) {
+              tmem_ld8(ty + (cc + 1) * 8, ev[(cc + 1) % NB]);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+              const uint64_t ey = f2_pack(__uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
+              const uint64_t dd = f2_pack(__uint_as_float(v[cc * 8 + j]), __uint_as_float(v[cc * 8 + j + 1]));
+              float x0, x1;
+              f2_unpack(f2_fma(dd, kc2, nc), x0, x1);
+              sqp = f2_fma(ey, f2_pack(ex2(x0), ex2(x1)), sqp);
+              ap = f2_fma(ey, dd, ap);
+            }
+            if (NB == 2 && cc + 1 < 8) tc_wait_ld8(ev[(cc + 1) % NB]);
           }
-          if (NB == 2 && cc + 1 < 8) tc_wait_ld8(ev[(cc + 1) % NB]);
         }
         float sq0, sq1, a0, a1;
         f2_unpack(sqp, sq0, sq1);
@@ -604,6 +702,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           xo[1] = sy;
           xo[2] = sq0 + sq1;
           xo[3] = a0 + a1;
+          xs[8 + par] = csh;
           __syncwarp();
           if (lane == 0) mbar_arrive(&xb[2 + par]);
         } else {
@@ -613,7 +712,19 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
               outp[0] = Mt * kOpUnscale;
               outp[SB_BM] = sy + xo[1];
             }
-            outp[(size_t)(2 + 2 * step) * SB_BM] = (sq0 + sq1) + xo[2];
+            // S_q of the row: the plain sum when neither half is shifted (the
+            // usual case); else the halves at a common shift, stored as the
+            // value if it fits below 2^120 and otherwise as minus its log2
+            // (S_q > 0, so a negative entry is unambiguous)
+            const float c1 = xs[8 + par];
+            float sq = (sq0 + sq1) + xo[2];
+            if (csh != 0.f || c1 != 0.f) {
+              const float ct = fmaxf(csh, c1);
+              const float s = pow2i(csh - ct) * (sq0 + sq1) + pow2i(c1 - ct) * xo[2];
+              const float l2 = log2f(s) + ct;
+              sq = l2 < 120.f ? exp2f(l2) : -l2;
+            }
+            outp[(size_t)(2 + 2 * step) * SB_BM] = sq;
             outp[(size_t)(3 + 2 * step) * SB_BM] = ((a0 + a1) + xo[3]) * kOpUnscale;
           }
         }
@@ -629,8 +740,13 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
 }
 
 // ---------------------------------------------------------------- merge and final
+// Per token: KL_t = log(S_q / S_y) - A / S_y from the output tiles' partials,
+// each tile's sums rescaled to the token's overall maximum M (fp64); an S_q
+// partial stored as minus its log2 (it would not fit fp32) is 2^-v. MSE
+// (objective 1): the tiles' sums of d^2, x 2^-16 / m.
 __global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict__ part, int n_ot, int P, int64_t N,
-                                                        int n_tt, double* __restrict__ kl_part) {
+                                                        int n_tt, int objective, int64_t m,
+                                                        double* __restrict__ kl_part) {
   extern __shared__ float s_f[];  // [n_ot][128] scale factors (one partial set per output tile)
   constexpr int QB = 8;  // candidates per pass
   __shared__ double red[4][QB];
@@ -638,13 +754,16 @@ __global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict_
   const int F = 2 + 2 * P;
   const bool valid = (int64_t)tt * SB_BM + r < N;
   const float* base = part + (size_t)tt * n_ot * F * SB_BM + r;
+  const bool mse = objective == 1;
   float M = -3.0e38f;
-  for (int og = 0; og < n_ot; ++og) M = fmaxf(M, base[(size_t)og * F * SB_BM]);
   double Sy = 0.0;
-  for (int og = 0; og < n_ot; ++og) {
-    const float f = exp2f((base[(size_t)og * F * SB_BM] - M) * kLog2e);
-    s_f[og * SB_BM + r] = f;
-    Sy += (double)base[(size_t)og * F * SB_BM + SB_BM] * (double)f;
+  if (!mse) {
+    for (int og = 0; og < n_ot; ++og) M = fmaxf(M, base[(size_t)og * F * SB_BM]);
+    for (int og = 0; og < n_ot; ++og) {
+      const float f = exp2f((base[(size_t)og * F * SB_BM] - M) * kLog2e);
+      s_f[og * SB_BM + r] = f;
+      Sy += (double)base[(size_t)og * F * SB_BM + SB_BM] * (double)f;
+    }
   }
   // candidates in blocks of QB: one pass over the output tiles loads 2 QB
   // independent values per tile (the sums run over the tiles in order, as
@@ -655,19 +774,21 @@ __global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict_
 #pragma unroll
     for (int j = 0; j < QB; ++j) sq[j] = a[j] = 0.0;
     for (int og = 0; og < n_ot; ++og) {
-      const double f = s_f[og * SB_BM + r];
+      const double f = mse ? 1.0 : (double)s_f[og * SB_BM + r];
       const float* bq = base + ((size_t)og * F + 2 + 2 * q0) * SB_BM;
 #pragma unroll
       for (int j = 0; j < QB; ++j)
         if (j < nq) {
-          sq[j] += (double)bq[(size_t)(2 * j) * SB_BM] * f;
+          const float v = bq[(size_t)(2 * j) * SB_BM];
+          sq[j] += (v >= 0.f ? (double)v : exp2(-(double)v)) * f;
           a[j] += (double)bq[(size_t)(2 * j + 1) * SB_BM] * f;
         }
     }
 #pragma unroll
     for (int j = 0; j < QB; ++j)
       if (j < nq) {
-        double kl = valid ? (log(sq[j] / Sy) - a[j] / Sy) : 0.0;
+        double kl = 0.0;
+        if (valid) kl = mse ? sq[j] * (1.0 / 65536.0) / (double)m : (log(sq[j] / Sy) - a[j] / Sy);
         kl = warp_sum(kl);
         if ((r & 31) == 0) red[r >> 5][j] = kl;
       }
@@ -716,10 +837,32 @@ __global__ void sba_final_kernel(const double* __restrict__ kl_part, int n_tt, i
 // Workspace: [prepared operands: Wb, E0, Dp, Dm, X as fp16][search: partials, KL parts].
 // The prepared region depends only on W and X, so it can be filled early.
 struct SbaPlan {
-  int k, P, ksplit, n_tt, n_tp, n_ot, stages, nA, nD;
-  size_t off_wb, off_e0, off_dp, off_dm, off_xc, off_part, off_klp, total;
+  int k, P, ksplit, nsub, npad, nbox, n_tt, n_tp, n_ot, stages;
+  size_t off_wb, off_e0, off_dp, off_dm, off_xc, off_split, off_part, off_klp, total;
   size_t smem;
 };
+
+// Box selection (bf16 X): column energies of W (all rows) and of X (its first
+// kSelTokens tokens), then per 64-column box the score sum_j |x_j|^2 |w_j|^2, an
+// estimate of the variance that fp16 rounding of the box's weight-side operands
+// adds to the outputs. Boxes are taken in descending score until what is left
+// is at most kSelRemainder of the total; those boxes are split into hi and lo.
+constexpr int64_t kSelTokens = 16384;
+constexpr int kSelRowsX = 128;
+constexpr double kSelRemainder = 1.0 / 32.0;
+// rows of W per block: 32, more for very tall W so the grid stays within 32768 row blocks
+static int64_t sel_rows_w(int64_t m) {
+  const int64_t r = (m + 32767) / 32768;
+  return r > 32 ? r : 32;
+}
+static int sel_row_blocks_w(int64_t m) { return (int)((m + sel_rows_w(m) - 1) / sel_rows_w(m)); }
+static int sel_row_blocks_x(int64_t N) {
+  const int64_t t = N < kSelTokens ? N : kSelTokens;
+  return (int)((t + kSelRowsX - 1) / kSelRowsX);
+}
+static size_t sel_bytes(int64_t m, int64_t n, int64_t N) {
+  return ((size_t)(sel_row_blocks_w(m) + sel_row_blocks_x(N)) * n + n) * sizeof(double);
+}
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -728,22 +871,30 @@ SbaPlan sba_plan(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
   pl.k = (int)(n / group);
   pl.P = pl.k / 2 + 1;
   pl.ksplit = xdtype == 1 ? 1 : 2;
+  pl.nsub = xdtype == 1 ? 2 : 3;
+  pl.npad = (int)((n + SB_BK - 1) / SB_BK * SB_BK);
+  pl.nbox = pl.npad / SB_BK;
   pl.n_tt = (int)((N + SB_BM - 1) / SB_BM);
   pl.n_ot = (int)((m + SB_BN - 1) / SB_BN);
   pl.n_tp = (pl.n_tt + 1) / 2;
-  pl.nA = (int)((n + SB_BK - 1) / SB_BK) * pl.ksplit;
-  pl.nD = 2 * (group >= 64 ? group / 64 : 1) * pl.ksplit;
-  const size_t wbytes = (size_t)m * n * 2;
+  const size_t wbytes = (size_t)m * 2 * pl.npad * 2;  // hi and lo halves of npad columns each
   size_t off = 0;
   pl.off_wb = off; off = align256(off + wbytes);
   pl.off_e0 = off; off = align256(off + wbytes);
   pl.off_dp = off; off = align256(off + wbytes);
   pl.off_dm = off; off = align256(off + wbytes);
   pl.off_xc = off; off = align256(off + (size_t)N * pl.ksplit * n * 2);
-  pl.off_part = off; off = align256(off + (size_t)pl.n_tt * pl.n_ot * (2 + 2 * pl.P) * SB_BM * sizeof(float));
+  pl.off_split = off; off = align256(off + (size_t)pl.nbox);
+  pl.off_part = off;
+  {
+    const size_t partials = (size_t)pl.n_tt * pl.n_ot * (2 + 2 * pl.P) * SB_BM * sizeof(float);
+    const size_t sel = sel_bytes(m, n, N);  // the selection's scratch, before the partials exist
+    off = align256(off + (partials > sel ? partials : sel));
+  }
   pl.off_klp = off; off = align256(off + (size_t)pl.P * pl.n_tt * sizeof(double));
   pl.total = off;
-  const size_t fixed = 1024 + 512 + 256 + (size_t)(pl.k + 4) * 4 + 64 + 2 * 128 * 8 * sizeof(float);
+  const size_t fixed = 1024 + 512 + 256 + (size_t)(pl.k + 4) * 4 + 64 + 2 * 128 * 12 * sizeof(float) +
+                       (size_t)3 * pl.nbox * 2 + (size_t)((pl.nbox + 15) & ~15) + 16;
   int st = 3;
   while (st > 2 && fixed + (size_t)st * SB_STAGE > 227 * 1024) --st;
   pl.stages = st;
@@ -765,7 +916,7 @@ size_t sba_search_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group) 
   return pl.total - pl.off_part;
 }
 
-// The weight-side fp16 operands (RTN at b-1, b, b+1) into the prepared region
+// The weight-side fp16 hi/lo operands (RTN at b-1, b, b+1) into the prepared region
 // (pw: sba_prep_bytes). bps caps the resident blocks per SM: a small cap
 // leaves room on every SM for kernels that run beside these grid-stride loops
 // on other streams.
@@ -777,16 +928,21 @@ cudaError_t launch_sba_prep_w(const float* W, int64_t m, int64_t n, int64_t N, i
   __half* E0 = reinterpret_cast<__half*>(pw + pl.off_e0);
   __half* Dp = reinterpret_cast<__half*>(pw + pl.off_dp);
   __half* Dm = reinterpret_cast<__half*>(pw + pl.off_dm);
+  if (pl.npad != n) {  // the columns between n and npad of both halves must read as zero
+    cudaError_t e = cudaMemsetAsync(pw + pl.off_wb, 0, pl.off_xc - pl.off_wb, s);
+    if (e != cudaSuccess) return e;
+  }
   const int64_t total4 = m * n / 4;              // n is a multiple of 32
+  const int64_t n4 = n / 4, rs2 = 2 * (int64_t)pl.npad / 4, lo2 = pl.npad / 4;
   int pgrid = (int)((total4 + 255) / 256);        // 8 warps x 32 float4 per block and pass
   if (pgrid > num_sms * bps) pgrid = num_sms * bps;
   const float4* W4 = reinterpret_cast<const float4*>(W);
   uint2 *b0 = reinterpret_cast<uint2*>(Wb), *b1 = reinterpret_cast<uint2*>(E0), *b2 = reinterpret_cast<uint2*>(Dp),
         *b3 = reinterpret_cast<uint2*>(Dm);
   switch (group) {
-    case 32: sba_prep_kernel<32><<<pgrid, 256, 0, s>>>(W4, total4, avg_bits, b0, b1, b2, b3, st); break;
-    case 64: sba_prep_kernel<64><<<pgrid, 256, 0, s>>>(W4, total4, avg_bits, b0, b1, b2, b3, st); break;
-    case 128: sba_prep_kernel<128><<<pgrid, 256, 0, s>>>(W4, total4, avg_bits, b0, b1, b2, b3, st); break;
+    case 32: sba_prep_kernel<32><<<pgrid, 256, 0, s>>>(W4, total4, n4, rs2, lo2, avg_bits, b0, b1, b2, b3, st); break;
+    case 64: sba_prep_kernel<64><<<pgrid, 256, 0, s>>>(W4, total4, n4, rs2, lo2, avg_bits, b0, b1, b2, b3, st); break;
+    case 128: sba_prep_kernel<128><<<pgrid, 256, 0, s>>>(W4, total4, n4, rs2, lo2, avg_bits, b0, b1, b2, b3, st); break;
     default: return cudaErrorInvalidValue;
   }
   count_launches(1);
@@ -812,6 +968,107 @@ cudaError_t launch_sba_prep_x(const void* X, int64_t m, int64_t n, int64_t N, in
   return cudaGetLastError();
 }
 
+// Column sums of squares: blockIdx.y < rbw covers rows_w rows of W, the rest
+// kSelRowsX tokens of X (bf16); each thread 4 adjacent columns. Fixed-order
+// partials [row block][column], summed in order by sel_score_kernel.
+__global__ void sel_colsq_kernel(const float* __restrict__ W, int64_t m, int64_t n, int64_t rows_w,
+                                 const uint16_t* __restrict__ X, int64_t T0, int rbw, double* __restrict__ part) {
+  const int64_t col = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (col >= n) return;
+  const int rb = blockIdx.y;
+  double a[4] = {0.0, 0.0, 0.0, 0.0};
+  if (rb < rbw) {
+    const int64_t r0 = (int64_t)rb * rows_w, r1 = (r0 + rows_w < m) ? r0 + rows_w : m;
+    for (int64_t r = r0; r < r1; ++r) {
+      const float4 v = *reinterpret_cast<const float4*>(W + r * n + col);
+      a[0] += (double)v.x * v.x; a[1] += (double)v.y * v.y; a[2] += (double)v.z * v.z; a[3] += (double)v.w * v.w;
+    }
+  } else {
+    const int64_t r0 = (int64_t)(rb - rbw) * kSelRowsX, r1 = (r0 + kSelRowsX < T0) ? r0 + kSelRowsX : T0;
+    for (int64_t r = r0; r < r1; ++r) {
+      const uint2 v = *reinterpret_cast<const uint2*>(X + r * n + col);
+      const float x0 = __uint_as_float(v.x << 16), x1 = __uint_as_float(v.x & 0xFFFF0000u);
+      const float x2 = __uint_as_float(v.y << 16), x3 = __uint_as_float(v.y & 0xFFFF0000u);
+      a[0] += (double)x0 * x0; a[1] += (double)x1 * x1; a[2] += (double)x2 * x2; a[3] += (double)x3 * x3;
+    }
+  }
+  double* o = part + (int64_t)rb * n + col;
+  o[0] = a[0]; o[1] = a[1]; o[2] = a[2]; o[3] = a[3];
+}
+
+__global__ void sel_score_kernel(const double* __restrict__ part, int rbw, int rbx, int64_t n,
+                                 double* __restrict__ score) {
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= n) return;
+  double w = 0.0, x = 0.0;
+  for (int r = 0; r < rbw; ++r) w += part[(int64_t)r * n + j];
+  for (int r = 0; r < rbx; ++r) x += part[(int64_t)(rbw + r) * n + j];
+  score[j] = w * x;
+}
+
+// One block of 1024 threads, nbox <= 1024: box scores, their stable descending
+// rank, the shortest prefix of the ranking that leaves at most `rem` of the
+// total, flags for the boxes in it.
+__global__ void sel_pick_kernel(const double* __restrict__ score, int64_t n, int nbox, double rem,
+                                uint8_t* __restrict__ split) {
+  __shared__ double s_box[1024], s_sorted[1024];
+  __shared__ int s_keep;
+  const int b = threadIdx.x;
+  double v = 0.0;
+  if (b < nbox)
+    for (int64_t j = (int64_t)b * 64; j < (int64_t)b * 64 + 64 && j < n; ++j) v += score[j];
+  if (b < nbox) s_box[b] = v;
+  __syncthreads();
+  int rank = 0;
+  if (b < nbox) {
+    for (int o = 0; o < nbox; ++o) rank += (s_box[o] > v || (s_box[o] == v && o < b)) ? 1 : 0;
+    s_sorted[rank] = v;
+  }
+  __syncthreads();
+  if (b == 0) {
+    double total = 0.0;
+    for (int i = 0; i < nbox; ++i) total += s_sorted[i];
+    double left = total;
+    int keep = 0;
+    while (keep < nbox && left > rem * total) left -= s_sorted[keep++];
+    s_keep = keep;
+  }
+  __syncthreads();
+  if (b < nbox) split[b] = rank < s_keep ? 1 : 0;
+}
+
+// The split flags into the prepared region (pw), from W and X (bf16: the first
+// kSelTokens tokens), with the search region (sw) as scratch. precision 1: every
+// box split. fp32 X needs no flags (every box is taken in three parts).
+cudaError_t launch_sba_select(const float* W, const void* X, int64_t m, int64_t n, int64_t N, int xdtype, int group,
+                              int precision, uint8_t* pw, uint8_t* sw, cudaStream_t s) {
+  const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
+  uint8_t* flags = pw + pl.off_split;
+  if (xdtype != 1) return cudaSuccess;
+  if (pl.nbox > 1024) return cudaErrorInvalidValue;
+  if (precision == 1) {
+    count_launches(0);
+    return cudaMemsetAsync(flags, 1, (size_t)pl.nbox, s);
+  }
+  const int rbw = sel_row_blocks_w(m), rbx = sel_row_blocks_x(N);
+  const int64_t T0 = N < kSelTokens ? N : kSelTokens;
+  double* part = reinterpret_cast<double*>(sw);
+  double* score = part + (size_t)(rbw + rbx) * n;
+  sel_colsq_kernel<<<dim3((unsigned)((n / 4 + 255) / 256), (unsigned)(rbw + rbx)), 256, 0, s>>>(
+      W, m, n, sel_rows_w(m), static_cast<const uint16_t*>(X), T0, rbw, part);
+  sel_score_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, rbw, rbx, n, score);
+  sel_pick_kernel<<<1, 1024, 0, s>>>(score, n, pl.nbox, kSelRemainder, flags);
+  count_launches(3);
+  return cudaGetLastError();
+}
+
+// Where the split flags sit in the prepared region, and how many there are.
+size_t sba_split_offset(int64_t m, int64_t n, int64_t N, int xdtype, int group, int* nbox) {
+  const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
+  *nbox = pl.nbox;
+  return pl.off_split;
+}
+
 size_t sba_yd_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
   const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
   return (size_t)pl.n_tt * pl.n_ot * 2 * SB_BN * SB_BM * sizeof(float);
@@ -821,41 +1078,57 @@ size_t sba_yd_bytes(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
 // (pw) and the search region (sw).
 template <int MODE>
 static cudaError_t launch_score(const SbaPlan& pl, int64_t m, int64_t n, int64_t N, int group, const int32_t* order,
-                                const uint8_t* pw, uint8_t* sw, float* yd, int tp0, int tp1, DevStatus* st,
-                                int num_sms, cudaStream_t s, cudaEvent_t* kev) {
+                                int objective, const uint8_t* pw, uint8_t* sw, float* yd, int tp0, int tp1,
+                                DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev) {
   if (pl.k > SB_MAX_K || tp0 < 0 || tp1 > pl.n_tp || tp1 < tp0) return cudaErrorInvalidValue;
   if (tp1 == tp0) return cudaSuccess;
   SbaTmaps tm;
   bool ok = make_tmap_f16(&tm.x, pw + pl.off_xc, (uint64_t)(n * pl.ksplit), (uint64_t)N, SB_BK, SB_BM);
-  ok = ok && make_tmap_f16(&tm.wb, pw + pl.off_wb, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
-  ok = ok && make_tmap_f16(&tm.e0, pw + pl.off_e0, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
-  ok = ok && make_tmap_f16(&tm.dp, pw + pl.off_dp, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
-  ok = ok && make_tmap_f16(&tm.dm, pw + pl.off_dm, (uint64_t)n, (uint64_t)m, SB_BK, SB_BN);
+  const uint64_t wcols = 2 * (uint64_t)pl.npad;  // hi | lo
+  ok = ok && make_tmap_f16(&tm.wb, pw + pl.off_wb, wcols, (uint64_t)m, SB_BK, SB_BN);
+  ok = ok && make_tmap_f16(&tm.e0, pw + pl.off_e0, wcols, (uint64_t)m, SB_BK, SB_BN);
+  ok = ok && make_tmap_f16(&tm.dp, pw + pl.off_dp, wcols, (uint64_t)m, SB_BK, SB_BN);
+  ok = ok && make_tmap_f16(&tm.dm, pw + pl.off_dm, wcols, (uint64_t)m, SB_BK, SB_BN);
   if (!ok) return cudaErrorInvalidValue;
   SbaParams p;
-  p.N = N; p.m = m; p.n = n; p.g = group; p.k = pl.k; p.P = pl.P; p.ksplit = pl.ksplit;
-  p.n_tt = pl.n_tt; p.n_tp = tp1 - tp0; p.n_ot = pl.n_ot; p.stages = pl.stages; p.nA = pl.nA; p.nD = pl.nD;
+  p.N = N; p.m = m; p.n = n; p.npad = pl.npad; p.g = group; p.k = pl.k; p.P = pl.P; p.ksplit = pl.ksplit;
+  p.nsub = pl.nsub; p.nbox = pl.nbox; p.split = pw + pl.off_split;
+  p.n_tt = pl.n_tt; p.n_tp = tp1 - tp0; p.n_ot = pl.n_ot; p.stages = pl.stages;
   p.order = order; p.part = reinterpret_cast<float*>(sw); p.yd = yd; p.tp0 = tp0; p.st = st;
+  // A test can shorten one wait (the epilogue's wait for its accumulator) with
+  // SLIM_TEST_ACC_WAIT_NS, to check that a wait that runs out returns
+  // SLIM_ETIMEOUT and leaves the device usable. Nothing else reads it.
+  p.acc_wait_ns = kWaitLimitNs;
+  if (const char* t = std::getenv("SLIM_TEST_ACC_WAIT_NS")) {
+    const unsigned long long v = std::strtoull(t, nullptr, 10);
+    if (v > 0 && v < kWaitLimitNs) p.acc_wait_ns = v;
+  }
   static std::atomic<uint64_t> attr{0};
   uint64_t bit = 0;
   if (attr_pending(attr, bit)) {  // the plan's shared memory never exceeds this bound
-    cudaError_t e = cudaFuncSetAttribute(sba_score_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(sba_score_kernel<MODE, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          227 * 1024);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(sba_score_kernel<MODE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     if (e != cudaSuccess) return e;
     attr.fetch_or(bit);
   }
   const int units = p.n_tp * pl.n_ot;
   const int grid = units < num_sms ? units : num_sms;
   if (kev) cudaEventRecord(kev[0], s);
-  sba_score_kernel<MODE><<<grid, SB_THREADS, pl.smem, s>>>(tm, p);
+  if (objective == 1)
+    sba_score_kernel<MODE, 1><<<grid, SB_THREADS, pl.smem, s>>>(tm, p);
+  else
+    sba_score_kernel<MODE, 0><<<grid, SB_THREADS, pl.smem, s>>>(tm, p);
   if (kev) cudaEventRecord(kev[1], s);
   count_launches(1);
   return cudaGetLastError();
 }
 
 // Per-token KL from the partials, its means over tokens, p* and the bits.
-static cudaError_t launch_merge_final(const SbaPlan& pl, int64_t N, int avg_bits, const int32_t* order, double* kl,
-                                      int32_t* p_star, uint8_t* bits, uint8_t* sw, cudaStream_t s) {
+static cudaError_t launch_merge_final(const SbaPlan& pl, int64_t m, int64_t N, int avg_bits, const int32_t* order,
+                                      int objective, double* kl, int32_t* p_star, uint8_t* bits, uint8_t* sw,
+                                      cudaStream_t s) {
   float* part = reinterpret_cast<float*>(sw);
   double* klp = reinterpret_cast<double*>(sw + (pl.off_klp - pl.off_part));
   const size_t msmem = (size_t)pl.n_ot * SB_BM * sizeof(float);
@@ -863,7 +1136,7 @@ static cudaError_t launch_merge_final(const SbaPlan& pl, int64_t N, int avg_bits
     cudaError_t e = cudaFuncSetAttribute(sba_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
     if (e != cudaSuccess) return e;
   }
-  sba_merge_kernel<<<pl.n_tt, SB_BM, msmem, s>>>(part, pl.n_ot, pl.P, N, pl.n_tt, klp);
+  sba_merge_kernel<<<pl.n_tt, SB_BM, msmem, s>>>(part, pl.n_ot, pl.P, N, pl.n_tt, objective, m, klp);
   sba_final_kernel<<<1, 256, 0, s>>>(klp, pl.n_tt, pl.P, N, order, pl.k, avg_bits, kl, p_star, bits);
   count_launches(2);
   return cudaGetLastError();
@@ -872,48 +1145,52 @@ static cudaError_t launch_merge_final(const SbaPlan& pl, int64_t N, int avg_bits
 // Scoring, merge and final selection on the prepared operands (pw) with the
 // search region (sw: sba_search_bytes) for the partial sums.
 cudaError_t launch_sba_search(int64_t m, int64_t n, int xdtype, int64_t N, int group, int avg_bits,
-                              const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, const uint8_t* pw,
-                              uint8_t* sw, DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev) {
+                              const int32_t* order, int objective, double* kl, int32_t* p_star, uint8_t* bits,
+                              const uint8_t* pw, uint8_t* sw, DevStatus* st, int num_sms, cudaStream_t s,
+                              cudaEvent_t* kev) {
   const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
-  cudaError_t e = launch_score<kSbaAll>(pl, m, n, N, group, order, pw, sw, nullptr, 0, pl.n_tp, st, num_sms, s, kev);
+  cudaError_t e = launch_score<kSbaAll>(pl, m, n, N, group, order, objective, pw, sw, nullptr, 0, pl.n_tp, st,
+                                        num_sms, s, kev);
   if (e != cudaSuccess) return e;
-  return launch_merge_final(pl, N, avg_bits, order, kl, p_star, bits, sw, s);
+  return launch_merge_final(pl, m, N, avg_bits, order, objective, kl, p_star, bits, sw, s);
 }
 
 // Split search, first part: phase A for token-tile pairs [tp0, tp1) (pairs of
 // 128-token tiles); it needs only the prepared operands of those tokens.
 // Writes the pairs' phase-A partials into sw and their TMEM state into yd
 // (sba_yd_bytes).
-cudaError_t launch_sba_phase_a(int64_t m, int64_t n, int xdtype, int64_t N, int group, int tp0, int tp1,
-                               const uint8_t* pw, uint8_t* sw, float* yd, DevStatus* st, int num_sms,
+cudaError_t launch_sba_phase_a(int64_t m, int64_t n, int xdtype, int64_t N, int group, int objective, int tp0,
+                               int tp1, const uint8_t* pw, uint8_t* sw, float* yd, DevStatus* st, int num_sms,
                                cudaStream_t s) {
   const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
-  return launch_score<kSbaPhaseA>(pl, m, n, N, group, nullptr, pw, sw, yd, tp0, tp1, st, num_sms, s, nullptr);
+  return launch_score<kSbaPhaseA>(pl, m, n, N, group, nullptr, objective, pw, sw, yd, tp0, tp1, st, num_sms, s,
+                                  nullptr);
 }
 
 // Split search, second part, once every pair's phase A is in sw and yd: the
 // candidate steps, merge and final selection.
 cudaError_t launch_sba_steps(int64_t m, int64_t n, int xdtype, int64_t N, int group, int avg_bits,
-                             const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, const uint8_t* pw,
-                             uint8_t* sw, float* yd, DevStatus* st, int num_sms, cudaStream_t s) {
+                             const int32_t* order, int objective, double* kl, int32_t* p_star, uint8_t* bits,
+                             const uint8_t* pw, uint8_t* sw, float* yd, DevStatus* st, int num_sms, cudaStream_t s) {
   const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
   if (pl.P > 1) {
-    cudaError_t e = launch_score<kSbaSteps>(pl, m, n, N, group, order, pw, sw, yd, 0, pl.n_tp, st, num_sms, s,
-                                            nullptr);
+    cudaError_t e = launch_score<kSbaSteps>(pl, m, n, N, group, order, objective, pw, sw, yd, 0, pl.n_tp, st,
+                                            num_sms, s, nullptr);
     if (e != cudaSuccess) return e;
   }
-  return launch_merge_final(pl, N, avg_bits, order, kl, p_star, bits, sw, s);
+  return launch_merge_final(pl, m, N, avg_bits, order, objective, kl, p_star, bits, sw, s);
 }
 
 cudaError_t launch_sba(const float* W, int64_t m, int64_t n, const void* X, int xdtype, int64_t N, int group,
-                       int avg_bits, const int32_t* order, double* kl, int32_t* p_star, uint8_t* bits, uint8_t* ws,
-                       DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev) {
+                       int avg_bits, const int32_t* order, int objective, int precision, double* kl, int32_t* p_star,
+                       uint8_t* bits, uint8_t* ws, DevStatus* st, int num_sms, cudaStream_t s, cudaEvent_t* kev) {
   const SbaPlan pl = sba_plan(m, n, N, xdtype, group);
   cudaError_t e = launch_sba_prep_w(W, m, n, N, xdtype, group, avg_bits, ws, st, num_sms, 8, s);
   if (e == cudaSuccess) e = launch_sba_prep_x(X, m, n, N, xdtype, group, 0, N, ws, st, num_sms, 8, s);
+  if (e == cudaSuccess) e = launch_sba_select(W, X, m, n, N, xdtype, group, precision, ws, ws + pl.off_part, s);
   if (e != cudaSuccess) return e;
-  return launch_sba_search(m, n, xdtype, N, group, avg_bits, order, kl, p_star, bits, ws, ws + pl.off_part, st,
-                           num_sms, s, kev);
+  return launch_sba_search(m, n, xdtype, N, group, avg_bits, order, objective, kl, p_star, bits, ws,
+                           ws + pl.off_part, st, num_sms, s, kev);
 }
 
 }  // namespace slim

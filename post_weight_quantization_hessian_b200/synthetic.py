@@ -217,3 +217,30 @@ def sweep_spec(block: int, layer: int, N: int = CALIB_TOKENS) -> LayerSpec:
     return LayerSpec(name=f"llama7b_block{block}_{name}", m=m, n=n, N=N, x_dtype="bf16", group=128,
                      avg_bits=2, seed=1000 * block + layer, cluster_starts=scaled_cluster_starts(n),
                      n_x_outliers=8 if n == 4096 else 16)
+
+
+def device_layer(spec: LayerSpec, device="cuda", chunk_rows: int = 16384):
+    """W (float32 [m, n]) and X (bf16 [N, n]) of a layer drawn directly on the device
+    with torch's generator, seeded by spec.seed: the same recipe as make_weight /
+    make_activations (N(0, w_std^2) weights with the salient columns scaled,
+    N(0, 1) tokens with the outlier columns scaled, rounded once to bf16), but
+    another random stream. The 7B sweep uses it, where hundreds of layers with
+    gigabytes of tokens each would take hours to draw on the host; copy a
+    layer's tensors to the host to give the same values to the oracle.
+    """
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(spec.seed))
+    W = torch.randn((spec.m, spec.n), generator=g, device=device, dtype=torch.float32) * spec.w_std
+    cols = torch.from_numpy(salient_columns(spec)).to(device)
+    if cols.numel():
+        W[:, cols] *= spec.w_scale
+    X = torch.empty((spec.N, spec.n), dtype=torch.bfloat16, device=device)
+    ocols = torch.from_numpy(outlier_columns(spec)).to(device)
+    for r0 in range(0, spec.N, chunk_rows):
+        r1 = min(spec.N, r0 + chunk_rows)
+        x = torch.randn((r1 - r0, spec.n), generator=g, device=device, dtype=torch.float32)
+        if ocols.numel():
+            x[:, ocols] *= spec.x_scale
+        X[r0:r1] = x.to(torch.bfloat16)
+    return W, X

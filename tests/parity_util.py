@@ -9,12 +9,22 @@ Tolerances (stated once, used by every GPU test):
   H (fp32 X)     relative 1e-12 (fp64 accumulation of exact products)
   h, S           relative 1e-9 / 1e-12 on identical inputs (fp64, different
                  summation order and blocking)
-  KL_p           absolute 1e-4 (the target tolerance); observed deviations are
-                 printed (fp16 tensor-core operands, fp32 sums: 1e-6 to 7e-5 seen)
+  KL_p           absolute 2.5e-5 (KL_ATOL; the stated target is 1e-4). The
+                 weight-side tensor-core operands are fp16 hi/lo pairs (22
+                 significant bits), so what remains is the fp32 accumulation
+                 in tensor memory: over the longest chain (n/16 + (P-1) 2g/16
+                 K-steps, about 640 for the 13B up_proj at group 32) the
+                 truncating accumulator shrinks |d| by up to ~2e-5 relative,
+                 which moves KL by about twice that relative; emulated on an
+                 up_proj-shaped layer: 1.8e-5 of KL. KL values reach ~1.5.
+                 Observed deviations are printed.
   decisions      order, p*, tau index and codes are compared exactly; a
-                 difference is accepted only where the oracle's own relative gap
-                 between the two choices is below the stated threshold, i.e. the
-                 two are tied to within the GPU arithmetic's error.
+                 difference is accepted only where the oracle's own gap between
+                 the two choices is within what the GPU's measured error on
+                 that run could flip: for p*, twice the largest |dKL| measured
+                 on the same run; for the order, twice the largest relative
+                 deviation of the group saliences (S) on that run. Every such
+                 acceptance is printed.
 """
 from __future__ import annotations
 
@@ -24,7 +34,7 @@ import torch
 from oracle import slim_oracle as O
 from post_weight_quantization_hessian_b200 import synthetic as syn
 
-KL_ATOL = 1e-4
+KL_ATOL = 2.5e-5
 SYRK_SLICE_TOKENS = 16384
 
 
@@ -59,12 +69,16 @@ def order_ok(order_gpu, S_ref, rel=1e-6):
     return int(np.sum(og != O.salience_order(S_ref)))
 
 
-def pstar_ok(p_gpu, kl_ref, rel=1e-4):
+def pstar_ok(p_gpu, kl_ref, kl_gpu):
+    """p* must equal the oracle's, unless the oracle's own KL gap between the two is
+    at most twice the largest |dKL| of this run (a tie the GPU's error can flip)."""
     p_ref = int(np.argmin(kl_ref))
     if p_gpu == p_ref:
         return True
-    gap = (kl_ref[p_gpu] - kl_ref[p_ref]) / max(kl_ref[p_ref], 1e-300)
-    assert gap < rel, f"p* {p_gpu} vs oracle {p_ref}, oracle gap {gap:.3e}"
+    tol = 2.0 * float(np.abs(np.asarray(kl_gpu) - np.asarray(kl_ref)).max())
+    gap = kl_ref[p_gpu] - kl_ref[p_ref]
+    assert gap <= tol, f"p* {p_gpu} vs oracle {p_ref}, oracle gap {gap:.3e} > 2 max|dKL| {tol:.3e}"
+    print(f"p* near tie accepted: {p_gpu} vs {p_ref}, oracle gap {gap:.3e} <= {tol:.3e}")
     return False
 
 
@@ -105,12 +119,14 @@ def comparable_candidates(order_gpu, order_ref):
             if set(a[:p].tolist()) == set(b[:p].tolist()) and set(a[k - p:].tolist()) == set(b[k - p:].tolist())]
 
 
-def allocation_ok(bits_gpu, order_gpu, p_gpu, bits_ref, kl_ref, S_ref, avg_bits, kl_tol=2 * KL_ATOL, s_rel=1e-5):
+def allocation_ok(bits_gpu, order_gpu, p_gpu, bits_ref, kl_ref, S_ref, avg_bits, kl_tol, s_rel):
     """The GPU's allocation against the stored one. It must be the allocation its own order
     and p* define, and equal the stored one except where the stored values are near ties that
     the GPU's arithmetic can resolve either way: a p* whose stored KL is within kl_tol of the
     best, or groups swapped across a promote/demote boundary whose stored saliences differ by
-    less than s_rel. Returns '' when equal, else what differed."""
+    less than s_rel. The callers derive kl_tol and s_rel from the errors measured on the same
+    run (twice the largest |dKL|, twice the largest relative S deviation). Returns '' when
+    equal, else what differed (and prints it)."""
     bits_gpu = np.asarray(bits_gpu).astype(int)
     bits_ref = np.asarray(bits_ref).astype(int)
     kl_ref = np.asarray(kl_ref, dtype=np.float64)
@@ -119,7 +135,8 @@ def allocation_ok(bits_gpu, order_gpu, p_gpu, bits_ref, kl_ref, S_ref, avg_bits,
     p_ref = int(np.argmin(kl_ref))
     if p_gpu != p_ref:
         gap = kl_ref[p_gpu] - kl_ref[p_ref]
-        assert gap <= kl_tol, f"p* {p_gpu} vs stored {p_ref}: stored KL gap {gap:.3e}"
+        assert gap <= kl_tol, f"p* {p_gpu} vs stored {p_ref}: stored KL gap {gap:.3e} > {kl_tol:.3e}"
+        print(f"allocation: p* near tie accepted ({p_gpu} vs {p_ref}, stored gap {gap:.3e} <= {kl_tol:.3e})")
         return "p* (near tie)"
     if (bits_gpu == bits_ref).all():
         return ""
@@ -127,4 +144,5 @@ def allocation_ok(bits_gpu, order_gpu, p_gpu, bits_ref, kl_ref, S_ref, avg_bits,
     for c in diff:
         near = [o for o in diff if o != c and abs(S_ref[c] - S_ref[o]) <= s_rel * max(abs(S_ref[c]), abs(S_ref[o]))]
         assert near, f"group {c} has bits {bits_gpu[c]} vs stored {bits_ref[c]} with no near-tie partner"
+    print(f"allocation: near-tie swap accepted in groups {diff.tolist()} (relative S gap <= {s_rel:.3e})")
     return "near-tie swap"

@@ -39,7 +39,7 @@ def run_and_compare(s: syn.LayerSpec, h_rtol):
     mism = order_ok(g["order"], ref.S, rel=1e-5)               # vs the pipeline: near ties only
     sba_chain = O.sba_search(W, X, g["order"], s.group, s.avg_bits)
     assert np.abs(g["kl"] - sba_chain.kl).max() <= KL_ATOL
-    if pstar_ok(g["p_star"], sba_chain.kl):
+    if pstar_ok(g["p_star"], sba_chain.kl, g["kl"]):
         assert np.array_equal(g["bits"], sba_chain.bits.astype(np.uint8))
     assert g["bits"].astype(int).sum() == s.k * s.avg_bits
     sqc_chain = O.sqc_calibrate(W, g["h"], g["bits"], s.group, s.lam, s.n_tau)
@@ -84,9 +84,10 @@ def test_host_buffers_match_device_path(x_dtype):
     assert np.array_equal(bits, d["bits"].cpu().numpy())
 
 
-FULL_SIZE = [w for w in ("llama7b_q_proj_4096x4096", "llama7b_down_proj_4096x11008", "llama13b_up_proj_13824x5120",
-                          "llama13b_up_proj_13824x5120_g64", "llama13b_up_proj_13824x5120_g32")
-             if os.path.exists(os.path.join(os.path.dirname(__file__), "golden", f"{w}.json"))]
+# every benchmark layer shape; each needs its stored oracle values in tests/golden (a
+# missing file fails the test rather than dropping the case)
+FULL_SIZE = ["llama7b_q_proj_4096x4096", "llama7b_down_proj_4096x11008", "llama13b_up_proj_13824x5120",
+             "llama13b_up_proj_13824x5120_g64", "llama13b_up_proj_13824x5120_g32"]
 
 
 @pytest.mark.parametrize("workload", FULL_SIZE)
@@ -96,6 +97,8 @@ def test_full_size_sampled(workload):
     (b 3, levels 2/3/4), the 13B up_proj 13824x5120 at groups 128, 64 and 32. Full-N
     decisions are compared with the oracle's stored values (tests/golden)."""
     s = syn.WORKLOADS[workload]
+    gpath = os.path.join(os.path.dirname(__file__), "golden", f"{s.name}.json")
+    assert os.path.exists(gpath), f"stored oracle values missing: run tests/golden/make_golden.py --workload {s.name}"
     W, Xh, Wd, Xd = device_inputs(s)
     d = slim.slim_quantize_layer_ex(Wd, Xd, s.group, s.avg_bits, s.lam, s.n_tau)
     g = {k: (v.cpu().numpy() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
@@ -126,9 +129,9 @@ def test_full_size_sampled(workload):
     dev = np.abs(kl_s.cpu().numpy() - ref_s.kl).max()
     print(f"full-size subset KL max |dKL| {dev:.2e}; p* {int(p_s.item())} vs {ref_s.p_star}")
     assert dev <= KL_ATOL
-    pstar_ok(int(p_s.item()), ref_s.kl)
+    pstar_ok(int(p_s.item()), ref_s.kl, kl_s.cpu().numpy())
     # full-N decisions against the oracle's stored values (tests/golden, written by make_golden.py)
-    gold = json.load(open(os.path.join(os.path.dirname(__file__), "golden", f"{s.name}.json")))
+    gold = json.load(open(gpath))
     S_gold = np.array(gold["S"])
     # the truncating tensor-core accumulation scales H by up to hessian_bound; h and so
     # S inherit about twice that relative shift, nearly uniform across groups
@@ -140,20 +143,26 @@ def test_full_size_sampled(workload):
     kl_gold = np.array(gold["kl"])
     dkl = np.abs(np.asarray(g["kl"])[comp] - kl_gold[comp]).max()
     assert dkl <= KL_ATOL
-    how = allocation_ok(g["bits"], g["order"], int(g["p_star"]), gold["bits"], kl_gold, S_gold, s.avg_bits)
+    # near-tie allowances from this run's own measured errors; the S deviation is taken
+    # after removing the common factor that the truncating H accumulation introduces
+    s_ratio = np.asarray(g["S"]) / S_gold
+    s_rel = 2.0 * float(np.abs(s_ratio / np.median(s_ratio) - 1.0).max())
+    how = allocation_ok(g["bits"], g["order"], int(g["p_star"]), gold["bits"], kl_gold, S_gold, s.avg_bits,
+                        kl_tol=2.0 * dkl, s_rel=s_rel)
     print(f"full-size vs golden: order mismatches {mism} (near ties only), {len(comp)} of {len(kl_gold)} "
           f"candidates comparable, max |dKL| {dkl:.2e}, p* {g['p_star']} vs {gold['p_star']}, "
-          f"allocation {how or 'equal'}")
+          f"allocation {how or 'equal'}, S relative spread {s_rel / 2:.2e}")
     # full-N search: invariants
     kl = g["kl"]
     assert np.all(kl >= 0) and g["p_star"] == int(np.argmin(kl))
     b = g["bits"].astype(int)
     assert b.sum() == s.k * s.avg_bits
     assert (b == s.avg_bits + 1).sum() == (b == s.avg_bits - 1).sum() == g["p_star"]
-    # SQC on sampled rows with the GPU's h and bits
-    rows = np.sort(rng.choice(s.m, 64, replace=False))
-    ref_q = O.sqc_calibrate(W[rows], g["h"], g["bits"], s.group, s.lam, s.n_tau)
-    agree, tmis = compare_sqc(g["codes"][rows], g["scale"][rows], g["zero"][rows], g["tau_idx"][rows], ref_q,
-                              g["bits"], s.group, s.avg_bits)
+    # SQC on every row with the GPU's h and bits (SQC does not depend on N, so the
+    # whole layer is cheap for the oracle)
+    ref_q = O.sqc_calibrate(W, g["h"], g["bits"], s.group, s.lam, s.n_tau)
+    agree, tmis = compare_sqc(g["codes"], g["scale"], g["zero"], g["tau_idx"], ref_q, g["bits"], s.group,
+                              s.avg_bits)
+    print(f"full-size SQC on all {s.m} rows: packed-word agreement {agree:.6f}, tau mismatches {tmis}")
     assert agree >= 0.9999 and tmis == 0
     print(f"full-size {workload}: p* {g['p_star']}, KL {kl}, stage ms {g['stage_ms']}")

@@ -160,7 +160,7 @@ def test_sba_search(kw):
     dev = np.abs(kl - ref.kl).max()
     print(f"sba {kw}: KL {kl} ref {ref.kl} max|dKL| {dev:.2e} p* {int(p_star.item())}/{ref.p_star}")
     assert dev <= KL_ATOL
-    if pstar_ok(int(p_star.item()), ref.kl):
+    if pstar_ok(int(p_star.item()), ref.kl, kl):
         assert np.array_equal(bits.cpu().numpy(), ref.bits.astype(np.uint8))
     b = bits.cpu().numpy().astype(int)
     assert b.sum() == s.k * s.avg_bits
