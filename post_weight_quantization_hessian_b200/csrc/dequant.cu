@@ -30,20 +30,11 @@ constexpr int DG_WARPS = 4;
 constexpr int DG_MAXB = 8;
 
 // One warp per (batch row b, group c): x of the group's G columns as fp32
-// (bf16 widened exactly) into xf, their sum into xs[b][c]; block 0's first
-// thread also writes wstart[c] = (G / 32) * sum_{c' < c} bits[c'].
-__global__ void dg_prep_kernel(const uint8_t* __restrict__ bits, int k, int G, const void* __restrict__ x, int xdtype,
-                               int B, int64_t n, float* __restrict__ xf, float* __restrict__ xs,
-                               int* __restrict__ wstart) {
+// (bf16 widened exactly) into xf, their sum into xs[b][c].
+__global__ void dg_prep_kernel(int k, int G, const void* __restrict__ x, int xdtype, int B, int64_t n,
+                               float* __restrict__ xf, float* __restrict__ xs) {
   const int lane = threadIdx.x & 31;
   const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    int acc = 0;
-    for (int c = 0; c < k; ++c) {
-      wstart[c] = acc;
-      acc += (G / 32) * bits[c];
-    }
-  }
   if (e >= B * k) return;
   const int b = e / k, c = e - b * k;
   const int64_t base = (int64_t)b * n + (int64_t)c * G;
@@ -94,7 +85,7 @@ __device__ __forceinline__ void dg_group(const uint32_t (&buf)[G / 4], const flo
 template <int G>
 __global__ void __launch_bounds__(DG_WARPS * 32)
 dg_kernel(const uint32_t* __restrict__ codes, int64_t m, int64_t rw, const uint8_t* __restrict__ bits,
-          const int* __restrict__ wstart, const float* __restrict__ scale, const float* __restrict__ zero, int k,
+          const float* __restrict__ scale, const float* __restrict__ zero, int k,
           const float* __restrict__ xf, const float* __restrict__ xs, int B, int64_t n, int gps,
           float* __restrict__ part) {
   constexpr int NW = G / 4;  // words of a group at 8 bits, the widest
@@ -107,9 +98,15 @@ dg_kernel(const uint32_t* __restrict__ codes, int64_t m, int64_t rw, const uint8
 #pragma unroll
   for (int bb = 0; bb < DG_MAXB; ++bb) acc[bb] = 0.f;
   const uint32_t* rowp = codes + (valid ? row : 0) * rw;
-  for (int c = c0; c < c1; ++c) {
+  // word offset of group c0 in a row: (G / 32) * sum of the earlier groups' bits,
+  // summed by the warp's lanes (the same on every lane); later groups add theirs
+  int before = 0;
+  for (int c = lane; c < c0; c += 32) before += bits[c];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+  int ws = (G / 32) * before;
+  for (int c = c0; c < c1; ws += (G / 32) * bits[c], ++c) {
     const int b = bits[c];
-    const int ws = wstart[c];
     const int nw = (G / 32) * b;
     uint32_t buf[NW];
 #pragma unroll
@@ -165,7 +162,7 @@ size_t dg_workspace_bytes(int64_t m, int64_t n, int group, int64_t B, int num_sm
   const int k = (int)(n / group);
   const int ks = dg_splits(m, k, num_sms);
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
-  return al((size_t)B * n * 4) + al((size_t)B * k * 4) + al((size_t)k * 4) + al((size_t)ks * B * m * 4);
+  return al((size_t)B * n * 4) + al((size_t)B * k * 4) + al((size_t)ks * B * m * 4);
 }
 
 cudaError_t launch_dequant_gemv(const uint32_t* codes, const uint8_t* bits, const float* scale, const float* zero,
@@ -179,14 +176,13 @@ cudaError_t launch_dequant_gemv(const uint32_t* codes, const uint8_t* bits, cons
   auto al = [](size_t v) { return (v + 255) & ~size_t(255); };
   float* xf = reinterpret_cast<float*>(ws);
   float* xs = reinterpret_cast<float*>(ws + al((size_t)B * n * 4));
-  int* wstart = reinterpret_cast<int*>(ws + al((size_t)B * n * 4) + al((size_t)B * k * 4));
-  float* part = reinterpret_cast<float*>(ws + al((size_t)B * n * 4) + al((size_t)B * k * 4) + al((size_t)k * 4));
-  dg_prep_kernel<<<(B * k + 7) / 8, 256, 0, s>>>(bits, k, group, x, xdtype, B, n, xf, xs, wstart);
+  float* part = reinterpret_cast<float*>(ws + al((size_t)B * n * 4) + al((size_t)B * k * 4));
+  dg_prep_kernel<<<(B * k + 7) / 8, 256, 0, s>>>(k, group, x, xdtype, B, n, xf, xs);
   const dim3 grid((unsigned)(((m + 31) / 32 + DG_WARPS - 1) / DG_WARPS), (unsigned)ksr);
   switch (group) {
-    case 32: dg_kernel<32><<<grid, DG_WARPS * 32, 0, s>>>(codes, m, rw, bits, wstart, scale, zero, k, xf, xs, B, n, gps, part); break;
-    case 64: dg_kernel<64><<<grid, DG_WARPS * 32, 0, s>>>(codes, m, rw, bits, wstart, scale, zero, k, xf, xs, B, n, gps, part); break;
-    case 128: dg_kernel<128><<<grid, DG_WARPS * 32, 0, s>>>(codes, m, rw, bits, wstart, scale, zero, k, xf, xs, B, n, gps, part); break;
+    case 32: dg_kernel<32><<<grid, DG_WARPS * 32, 0, s>>>(codes, m, rw, bits, scale, zero, k, xf, xs, B, n, gps, part); break;
+    case 64: dg_kernel<64><<<grid, DG_WARPS * 32, 0, s>>>(codes, m, rw, bits, scale, zero, k, xf, xs, B, n, gps, part); break;
+    case 128: dg_kernel<128><<<grid, DG_WARPS * 32, 0, s>>>(codes, m, rw, bits, scale, zero, k, xf, xs, B, n, gps, part); break;
     default: return cudaErrorInvalidValue;
   }
   dg_reduce_kernel<<<(unsigned)((B * m + 255) / 256), 256, 0, s>>>(part, ksr, B, m, y);

@@ -515,17 +515,21 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
                   tc_mma_f16(ty1, a1 + 2 * k16, b0 + 2 * k16, idesc2, acc);
                 }
               } else if (dfull) {
+                // a step's update accumulates from zero (its own short chain); the
+                // epilogue adds it to d in registers
 #pragma unroll
                 for (int k16 = 0; k16 < 4; ++k16) {
-                  tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, 1u);
-                  tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, 1u);
+                  const uint32_t acc = (c > 0 || k16 > 0) ? 1u : 0u;
+                  tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, acc);
+                  tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, acc);
                 }
               } else {
                 Chunk ch;
                 chunk_at(p, geo, s_tab, c, ch);
                 for (int k16 = ch.k16_lo; k16 < ch.k16_hi; ++k16) {
-                  tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, 1u);
-                  tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, 1u);
+                  const uint32_t acc = (c > 0 || k16 > ch.k16_lo) ? 1u : 0u;
+                  tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, acc);
+                  tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, acc);
                 }
               }
               tc_commit(&empty[st]);
@@ -565,74 +569,31 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
       // this thread's 64 outputs of its token row in yd (e^(y - M); d at + 128 rows)
       float* ydp = p.yd + ((size_t)(have ? tt : 0) * p.n_ot + ot) * 2 * SB_BN * SB_BM + (size_t)(h * 64) * SB_BM + r;
       float Mt = 0.f;
+      // d of this thread's 64 outputs, kept in registers for the whole unit: phase A
+      // leaves d_0 in tensor memory, every later step its update alone, added here
+      // with round-to-nearest fp32 adds (the tensor core's accumulator truncates,
+      // which over the long chain of all steps would shrink |d| systematically)
+      uint32_t v[64];
       if (MODE == kSbaSteps) {
-        // phase A's TMEM contents back in place; the arrival on afree hands the
-        // slot to the first candidate step's MMAs (a unit's last step does not
-        // release the slot in this mode: this load does)
-        uint32_t v[64];
+        // phase A's e^(y - M) back in tensor memory and its d_0 into registers; the
+        // arrival on afree hands the slot to the first candidate step's MMAs (a
+        // unit's last step does not release the slot in this mode: this load does)
 #pragma unroll
         for (int j = 0; j < 64; ++j) v[j] = have ? __float_as_uint(ydp[(size_t)j * SB_BM]) : 0u;
         tmem_st32(ty, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
         tmem_st32(ty + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tc_wait_st();
 #pragma unroll
         for (int j = 0; j < 64; ++j) v[j] = have ? __float_as_uint(ydp[(size_t)(SB_BN + j) * SB_BM]) : 0u;
-        tmem_st32(td, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_st32(td + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        tc_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&afree[slot]);
       }
-      for (int step = s_lo; step < s_hi; ++step) {
-        if (!mbar_wait(&afull[slot], cnt & 1, abort_flag, p.st, 240 + slot, p.acc_wait_ns)) { ok = false; break; }
-        tc_fence_after();
-        uint32_t v[64];
-        float sy = 0.f;
-        if (step == 0) {
-          // y -> row maximum (both halves) -> e^(y - M) stored back in place of y
-          tmem_ld32(ty, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-          tmem_ld32(ty + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-          tc_wait_ld();
-          float mx = -3.0e38f;
-#pragma unroll
-          for (int j = 0; j < 64; ++j)
-            if (j < nvalid) mx = fmaxf(mx, __uint_as_float(v[j]));
-          xs[h ? 0 : 4] = mx;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&xb[h]);
-          if (!mbar_wait(&xb[h ^ 1], nunit & 1, abort_flag, p.st, 250 + slot)) { ok = false; break; }
-          mx = fmaxf(mx, xs[h ? 4 : 0]);
-          const float mb = -mx * kC1;
-#pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            const float ey = (j < nvalid) ? ex2(fmaf(__uint_as_float(v[j]), kC1, mb)) : 0.f;
-            sy += ey;
-            v[j] = __float_as_uint(ey);
-          }
-          tmem_st32(ty, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-          tmem_st32(ty + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-          if (MODE == kSbaPhaseA && have) {
-#pragma unroll
-            for (int j = 0; j < 64; ++j) ydp[(size_t)j * SB_BM] = __uint_as_float(v[j]);
-          }
-          tc_wait_st();
-          Mt = mx;
-        }
-        // this step's d to registers, then release the accumulator (except at the
-        // unit's last step: the next unit's first MMA overwrites e^(y - M))
-        tmem_ld32(td, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(td + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        tc_wait_ld();
-        if (MODE == kSbaPhaseA && have) {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) ydp[(size_t)(SB_BN + j) * SB_BM] = __uint_as_float(v[j]);
-        }
+      // The tail of every step: the sums of this step's d over the thread's 64
+      // outputs, the accumulator's release after the unit's last step, and the
+      // halves' exchange and partial stores. false: a wait gave up.
+      auto finish_step = [&](int step, float sy) -> bool {
         const bool last = step == s_hi - 1;
-        if (!last) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&afree[slot]);
-        }
         // Per-token sums over this thread's 64 outputs. KL: S_q = sum e^(y-M) e^d
         // and A = sum e^(y-M) d. MSE: the sum of d^2 (accumulator units, x 2^16).
         uint64_t sqp = 0, ap = 0;  // packed (even, odd column) sums
@@ -658,8 +619,8 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           const uint64_t kc2 = f2_pack(kC1, kC1), nc = f2_pack(-csh, -csh);
           // e^(y - M) in 8-column pieces. In the split launches the pieces are
           // double-buffered (the load of the next one is in flight while this one
-          // is consumed); the one-pass launch, whose step-0 code already holds
-          // more registers, loads them one at a time. Same arithmetic either way.
+          // is consumed); the one-pass launch loads them one at a time. Same
+          // arithmetic either way.
           constexpr int NB = MODE == kSbaAll ? 1 : 2;
           uint32_t ev[NB][8];
           if (NB == 2) {
@@ -706,7 +667,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           __syncwarp();
           if (lane == 0) mbar_arrive(&xb[2 + par]);
         } else {
-          if (!mbar_wait(&xb[2 + par], (cnt >> 1) & 1, abort_flag, p.st, 252 + slot)) { ok = false; break; }
+          if (!mbar_wait(&xb[2 + par], (cnt >> 1) & 1, abort_flag, p.st, 252 + slot)) return false;
           if (have) {
             if (step == 0) {
               outp[0] = Mt * kOpUnscale;
@@ -720,8 +681,8 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
             float sq = (sq0 + sq1) + xo[2];
             if (csh != 0.f || c1 != 0.f) {
               const float ct = fmaxf(csh, c1);
-              const float s = pow2i(csh - ct) * (sq0 + sq1) + pow2i(c1 - ct) * xo[2];
-              const float l2 = log2f(s) + ct;
+              const float s2 = pow2i(csh - ct) * (sq0 + sq1) + pow2i(c1 - ct) * xo[2];
+              const float l2 = log2f(s2) + ct;
               sq = l2 < 120.f ? exp2f(l2) : -l2;
             }
             outp[(size_t)(2 + 2 * step) * SB_BM] = sq;
@@ -729,6 +690,82 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           }
         }
         ++cnt;
+        return true;
+      };
+      // the accumulator's release once its contents are in registers (not after
+      // the unit's last step: the next unit's first MMA overwrites e^(y - M))
+      auto release_early = [&](int step) {
+        if (step != s_hi - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afree[slot]);
+        }
+      };
+      if (MODE != kSbaSteps) {
+        // step 0 (phase A): y -> row maximum (both halves) -> e^(y - M) stored back
+        // in place of y; then d_0 into registers
+        if (!mbar_wait(&afull[slot], cnt & 1, abort_flag, p.st, 240 + slot, p.acc_wait_ns)) { ok = false; break; }
+        tc_fence_after();
+        // y in 8-column pieces (the maximum, then e^(y - M) written back in
+        // place), so that no 64 registers besides d are needed
+        float sy = 0.f;
+        float mx = -3.0e38f;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t yv[8];
+          tmem_ld8(ty + cc * 8, yv);
+          tc_wait_ld8(yv);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (cc * 8 + j < nvalid) mx = fmaxf(mx, __uint_as_float(yv[j]));
+        }
+        xs[h ? 0 : 4] = mx;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xb[h]);
+        if (!mbar_wait(&xb[h ^ 1], nunit & 1, abort_flag, p.st, 250 + slot)) { ok = false; break; }
+        mx = fmaxf(mx, xs[h ? 4 : 0]);
+        const float mb = -mx * kC1;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t yv[8];
+          tmem_ld8(ty + cc * 8, yv);
+          tc_wait_ld8(yv);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float ey = (cc * 8 + j < nvalid) ? ex2(fmaf(__uint_as_float(yv[j]), kC1, mb)) : 0.f;
+            sy += ey;
+            yv[j] = __float_as_uint(ey);
+            if (MODE == kSbaPhaseA && have) ydp[(size_t)(cc * 8 + j) * SB_BM] = ey;
+          }
+          tmem_st8(ty + cc * 8, yv);
+        }
+        tc_wait_st();
+        Mt = mx;
+        tmem_ld32(td, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(td + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tc_wait_ld();
+        if (MODE == kSbaPhaseA && have) {
+#pragma unroll
+          for (int j = 0; j < 64; ++j) ydp[(size_t)(SB_BN + j) * SB_BM] = __uint_as_float(v[j]);
+        }
+        release_early(0);
+        if (!finish_step(0, sy)) { ok = false; break; }
+      }
+      for (int step = 1; step < s_hi; ++step) {
+        // candidate step: d += this step's update (round to nearest)
+        if (!mbar_wait(&afull[slot], cnt & 1, abort_flag, p.st, 240 + slot, p.acc_wait_ns)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t u[16];
+          tmem_ld16(td + 16 * q, u);
+          tc_wait_ld16(u);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            v[16 * q + j] = __float_as_uint(__fadd_rn(__uint_as_float(v[16 * q + j]), __uint_as_float(u[j])));
+        }
+        release_early(step);
+        if (!finish_step(step, 0.f)) { ok = false; break; }
       }
     }
   }
