@@ -262,12 +262,14 @@ def source_hash(*paths):
     return h.hexdigest()[:16]
 
 
-def traffic_record(kernel: str, src_hash: str):
+def traffic_record(kernel: str, workload: str, src_hash: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu summary
+    (profiles/traffic.json), or None when absent or taken on other source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f).get(kernel)
-    except (OSError, ValueError):
+            rec = json.load(f).get(kernel, {}).get(workload)
+    except (OSError, ValueError, AttributeError):
         return None
     if not rec or rec.get("source_hash") != src_hash:
         return None
@@ -321,18 +323,49 @@ def extra_kernels(spec, Wd, Xd, d, stages, flush, stream):
     del gws, H
     codes, scale, zero = d["codes"], d["scale"], d["zero"]
     rows = {}
+    # the call is microseconds long: it is timed from a CUDA graph of back-to-back calls, each
+    # on its own copy of the packed layer (copies together several times the L2), so the
+    # device time is measured without host launch gaps and every call reads from DRAM
+    layer_bytes = codes.numel() * 4 + 2 * scale.numel() * 4
+    ncopy = max(2, int(3 * 126e6 // layer_bytes) + 1)
+    copies = [(codes.clone(), scale.clone(), zero.clone()) for _ in range(ncopy)]
+    reps = max(24, ncopy)
     for B in (1, 8):
         x = torch.randn((B, n), device=Wd.device).to(torch.bfloat16)
-        y = torch.empty((B, m), dtype=torch.float32, device=Wd.device)
+        ys = [torch.empty((B, m), dtype=torch.float32, device=Wd.device) for _ in range(ncopy)]
         gws = torch.empty(slim._lib().slim_dequant_gemv_workspace_bytes(m, n, spec.group, B), dtype=torch.uint8,
                           device=Wd.device)
-        us = timed(lambda: slim.slim_dequant_gemv(codes, bits, scale, zero, spec.group, spec.avg_bits, x, y=y, ws=gws),
-                   20, flush, stream) * 1e3
-        byt = codes.numel() * 4 + 2 * scale.numel() * 4 + k + B * n * 2 + B * m * 4
+        side = torch.cuda.Stream(device=Wd.device)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for i in range(ncopy):
+                c_, s_, z_ = copies[i]
+                slim.slim_dequant_gemv(c_, bits, s_, z_, spec.group, spec.avg_bits, x, y=ys[i], ws=gws)
+        stream.wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(reps):
+                c_, s_, z_ = copies[i % ncopy]
+                slim.slim_dequant_gemv(c_, bits, s_, z_, spec.group, spec.avg_bits, x, y=ys[i % ncopy], ws=gws)
+        g.replay()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            b.synchronize()
+            ms.append(a.elapsed_time(b))
+        us = min(ms) * 1e3 / reps
+        del g
+        byt = layer_bytes + k + B * n * 2 + B * m * 4
         rows[f"batch{B}"] = {"us": us, "bytes": byt, "gbs": byt / (us * 1e-6) / 1e9,
                              "frac": byt / (us * 1e-6) / 1e9 / pk["hbm_gbs"]}
+    del copies
     out["dequant_gemv"] = dict(rows, note="y = x W_hat^T on the packed codes; bytes = codes + fp32 scale and "
-                                          "zero + bits + x + y, of the measured HBM copy bandwidth; L2 flushed")
+                                          "zero + bits + x + y, of the measured HBM copy bandwidth; device time "
+                                          f"per call from a CUDA graph of {reps} calls over {ncopy} copies of the layer")
     return out
 
 
@@ -426,7 +459,7 @@ def run_ours(args, spec, world, rank, local):
     src = source_hash("post_weight_quantization_hessian_b200/csrc/sba.cu",
                       "post_weight_quantization_hessian_b200/csrc/common.cuh")
     roofline = {"kernel": "sba_score_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic_record("sba_score_kernel", src),
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic_record("sba_score_kernel", spec.name, src),
                 "peak_kind": f"{pk_kind} bf16 dense burst (fp16 operands, same nominal rate)",
                 "flops_per_launch": flops, "ms_per_launch": sba_ms,
                 "flops_note": "executed: y and d_0 over K = n plus two groups per further candidate, "

@@ -810,6 +810,7 @@ __global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict_
     double sq[QB], a[QB];
 #pragma unroll
     for (int j = 0; j < QB; ++j) sq[j] = a[j] = 0.0;
+    bool shifted = false;
     for (int og = 0; og < n_ot; ++og) {
       const double f = mse ? 1.0 : (double)s_f[og * SB_BM + r];
       const float* bq = base + ((size_t)og * F + 2 + 2 * q0) * SB_BM;
@@ -817,9 +818,25 @@ __global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict_
       for (int j = 0; j < QB; ++j)
         if (j < nq) {
           const float v = bq[(size_t)(2 * j) * SB_BM];
-          sq[j] += (v >= 0.f ? (double)v : exp2(-(double)v)) * f;
+          shifted |= v < 0.f;
+          sq[j] += (double)v * f;
           a[j] += (double)bq[(size_t)(2 * j + 1) * SB_BM] * f;
         }
+    }
+    if (shifted) {
+      // rare: a partial stored as minus its log2 (see the scoring epilogue); the
+      // S_q sums of this pass again, decoding those entries
+#pragma unroll
+      for (int j = 0; j < QB; ++j) sq[j] = 0.0;
+      for (int og = 0; og < n_ot; ++og) {
+        const double f = mse ? 1.0 : (double)s_f[og * SB_BM + r];
+        const float* bq = base + ((size_t)og * F + 2 + 2 * q0) * SB_BM;
+        for (int j = 0; j < QB; ++j)
+          if (j < nq) {
+            const float v = bq[(size_t)(2 * j) * SB_BM];
+            sq[j] += (v >= 0.f ? (double)v : exp2(-(double)v)) * f;
+          }
+      }
     }
 #pragma unroll
     for (int j = 0; j < QB; ++j)
