@@ -200,23 +200,20 @@ __global__ void x_split_kernel(const float* __restrict__ X, int64_t N, int64_t n
 }
 
 // ---------------------------------------------------------------- scoring kernel
-constexpr int SB_BM = 128;        // tokens per tile (one CTA's TMEM lanes)
-constexpr int SB_BN = 128;        // outputs per tile
+constexpr int SB_BM = 128;        // tokens per tile (TMEM lanes)
+constexpr int SB_BN = 128;        // outputs per tile (one TMEM slot: y and d, 128 columns each)
 constexpr int SB_BK = 64;         // K elements per box (128 bytes of fp16)
 constexpr int SB_BOX = SB_BM * SB_BK * 2;  // 16 KB
-constexpr int SB_STAGE = 2 * SB_BOX;       // per CTA: its X box, its half of the weight-side rows
+constexpr int SB_STAGE = 4 * SB_BOX;       // X(token tile 0), X(token tile 1), B1, B2
 constexpr int SB_BAND = 16;                // token-tile pairs per raster band
 constexpr int SB_MAX_K = 1024;
-constexpr int SB_MAX_STAGES = 6;
-constexpr int SB_EPI_WARPS = 16;           // per CTA: four per TMEM lane quadrant, 32 columns each
+constexpr int SB_EPI_WARPS = 16;           // warps 2..9 read slot 0, warps 10..17 slot 1 (two per row)
 constexpr int SB_THREADS = 64 + 32 * SB_EPI_WARPS;
-constexpr int SB_XF = 32;                  // epilogue exchange fields per token row (shared, [field][row])
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kC1 = kLog2e * kOpUnscale;  // exponent scale for accumulator (x 2^8) units
 
 struct SbaTmaps {
-  CUtensorMap x, wb, e0;  // 64-column x 128-row boxes
-  CUtensorMap dp, dm;     // 64-column x 64-row boxes (each CTA of a pair loads half of an output tile)
+  CUtensorMap x, wb, e0, dp, dm;
 };
 
 struct SbaParams {
@@ -317,12 +314,6 @@ __device__ __forceinline__ void unit_decode(const SbaParams& p, int u, int& tp, 
   tp = p.tp0 + band_start + (r - ot * bc);
 }
 
-// Phase-A chunks of the next unit that go out after candidate step s of the
-// current one: [pa_mark(s - 1), pa_mark(s)), spreading phase A over the steps.
-__device__ __forceinline__ int pa_mark(int nA, int P, int s) {
-  return P > 1 ? (int)((int64_t)nA * s / (P - 1)) : nA;
-}
-
 // What one launch of the scoring kernel covers.
 enum SbaMode : int {
   kSbaAll = 0,     // phase A and every candidate step
@@ -341,7 +332,9 @@ __device__ __forceinline__ float pow2i(float k) {
   return k >= -126.f ? __int_as_float((127 + (int)k) << 23) : 0.f;
 }
 
-// Packed fp32 pairs (sm_100 f32x2 arithmetic): two output columns per instruction.
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): the epilogue handles two output
+// columns per instruction, which leaves more issue slots to the MMA thread on
+// the same SM sub-partition.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
@@ -355,9 +348,9 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 
@@ -368,61 +361,45 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// The scoring kernel runs on CTA pairs (clusters of two): one work unit is a
-// token-tile pair against one output tile, CTA r of the pair holding token tile
-// 2 tp + r. The tensor cores work on the pair as one unit (tcgen05 cta_group::2):
-// every MMA is M = 256 (each CTA's 128 tokens, from its own X box) and each
-// CTA holds half of the weight-side rows (phase A: the even CTA the Wb box, the
-// odd one the E0 box; a candidate step: 64 output rows of the Dp / Dm box
-// each), so a weight-side box crosses from L2 once per token-tile pair.
-// Each CTA's tensor memory has two regions of 256 columns, [y or e^(y-M) | d
-// or the step's update] of its token tile; consecutive units alternate
-// regions, and in the one-pass launch the next unit's phase A (tensor-bound)
-// is issued in slices between the current unit's candidate steps
-// (exponential-bound), so both run at once.
-//   warp 0      TMA producer (both CTAs; the copies of both count on the even
-//               CTA's stage barrier)
-//   warp 1      TMEM owner (512 columns, both CTAs) and, in the even CTA, the
-//               MMA issuer for the pair
-//   warps 2..17 epilogue (each CTA, its own tokens): four warps per TMEM lane
-//               quadrant, 32 outputs each. A thread adds each step's update to
-//               its d in registers (round to nearest) and releases the
-//               accumulator before computing, so the next candidate's MMA
-//               overlaps the exponentials; the four parts of a row combine
-//               their maximum and sums through shared memory.
+// One work unit is two token tiles (TMEM slots 0 and 1) against one output tile:
+// every weight-side box feeds both slots' MMAs, so per output tile the kernel
+// moves about a third fewer bytes than with one token tile.
+//   warp 0      TMA producer (4 boxes per phase-A chunk, 3 per delta chunk)
+//   warp 1      TMEM owner (512 columns) and MMA issuer: phase A as N = 256 MMAs
+//               (Wb and E0 boxes adjacent; y and d adjacent in TMEM), delta steps
+//               as N = 128 MMAs into d, in place
+//   warps 2..17 epilogue, eight per slot: two threads per token row, 64 columns
+//               each. A thread copies its d columns to registers and releases
+//               the accumulator before computing, so the next candidate's MMA
+//               overlaps the epilogue's exponentials; the two halves of a row
+//               combine their row maximum and sums through shared memory.
 // MODE splits the work in two launches (phase A does not depend on the
 // salience order, so it can run before the order exists): kSbaPhaseA also
-// stores each tile's e^(y - M) and d, exactly as they sit in tensor memory and
-// registers after phase A; kSbaSteps loads them back and continues with step 1,
-// so the two launches together compute bit for bit what one kSbaAll launch does.
+// stores each tile's e^(y - M) and d, exactly as they sit in TMEM after phase
+// A; kSbaSteps loads them back into TMEM and continues with step 1, so the
+// two launches together compute bit for bit what one kSbaAll launch does.
 template <int MODE, int OBJ>
 __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_constant__ SbaTmaps tm, SbaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * SB_STAGE);  // [S] (the even CTA's count both CTAs' copies)
-  uint64_t* empty = full + S;    // [S] the pair's MMAs are done with the stage
-  uint64_t* afull = empty + S;   // [2] the region's accumulator holds the next step
-  uint64_t* afree = afull + 2;   // [2] (even CTA) both epilogues are done reading the region
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * SB_STAGE);
+  uint64_t* empty = full + S;
+  uint64_t* afull = empty + S;   // [2] step accumulated in TMEM slot s
+  uint64_t* afree = afull + 2;   // [2] epilogue done reading slot s
   uint64_t* done = afree + 2;
-  uint64_t* xbm = done + 1;      // [4 quadrants] row maximum exchange
-  uint64_t* xbs = xbm + 4;       // [4 quadrants][2 parities] sums exchange
-  uint32_t* misc = reinterpret_cast<uint32_t*>(xbs + 8);  // TMEM address, abort flag, phase-A chunks
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-  int32_t* s_order = reinterpret_cast<int32_t*>(misc + 4);
-  float* s_x = reinterpret_cast<float*>(s_order + ((p.k + 3) & ~3));   // [SB_XF][128]
-  uint16_t* s_tab = reinterpret_cast<uint16_t*>(s_x + SB_XF * SB_BM);   // phase-A chunks: box << 2 | sub
-  uint8_t* s_split = reinterpret_cast<uint8_t*>(s_tab + 3 * p.nbox);    // [nbox]
+  uint64_t* xbar = done + 1;     // [8 row groups (slot, quadrant)][4]: max of half 0, max of half 1, sums x2
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(xbar + 32);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  int32_t* s_order = reinterpret_cast<int32_t*>(tslot + 2);
+  float* s_x = reinterpret_cast<float*>(s_order + ((p.k + 3) & ~3));  // [2 slots][128 rows][12]
+  uint16_t* s_tab = reinterpret_cast<uint16_t*>(s_x + 2 * 128 * 12);    // phase-A chunks: box << 2 | sub
+  uint8_t* s_split = reinterpret_cast<uint8_t*>(s_tab + 3 * p.nbox);   // [nbox]
+  int* s_na = reinterpret_cast<int*>(s_split + ((p.nbox + 15) & ~15));  // chunks of phase A
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_rank();
-  const int cl = blockIdx.x >> 1, ncl = gridDim.x >> 1;
-  // the launch's steps: [1, s_hi) after phase A (kSbaAll), phase A alone
-  // (kSbaPhaseA), [1, s_hi) from the stored state (kSbaSteps)
+  constexpr int s_lo = MODE == kSbaSteps ? 1 : 0;  // the launch's steps: [s_lo, s_hi)
   const int s_hi = MODE == kSbaPhaseA ? 1 : p.P;
-  // arrivals on afree[R] per unit: one per step but the last, one when the
-  // region is free again (in kSbaSteps the first is the state's load)
-  const uint32_t Pl = MODE == kSbaPhaseA ? 1u : (uint32_t)p.P;
   if (MODE != kSbaPhaseA)
     for (int c = threadIdx.x; c < p.k; c += blockDim.x) s_order[c] = p.order[c];
   for (int b = threadIdx.x; b < p.nbox; b += blockDim.x) s_split[b] = p.nsub == 3 ? 0 : (p.split[b] ? 1 : 0);
@@ -431,274 +408,199 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
     int c = 0;
     for (int b = 0; b < p.nbox; ++b)
       for (int u = 0; u < sub_count(p, s_split, b); ++u) s_tab[c++] = (uint16_t)(b << 2 | u);
-    misc[2] = (uint32_t)c;
+    *s_na = c;
     for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&afull[s], 1); mbar_init(&afree[s], 2 * SB_EPI_WARPS); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&afull[s], 1); mbar_init(&afree[s], SB_EPI_WARPS / 2); }
     mbar_init(done, 1);
-    for (int q = 0; q < 4; ++q) mbar_init(&xbm[q], 4);
-    for (int b = 0; b < 8; ++b) mbar_init(&xbs[b], 3);
+    for (int b = 0; b < 32; ++b) mbar_init(&xbar[b], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc_pair(misc, 512);
-  // both CTAs' barriers initialised and their TMEM allocated before either
-  // CTA touches the other's
-  tc_fence_before();
-  cluster_sync_all();
+  if (warp == 1) tmem_alloc(tslot, 512);
+  __syncthreads();
   tc_fence_after();
-  const uint32_t tbase = misc[0];
+  const uint32_t tbase = *tslot;
   const int units = p.n_tp * p.n_ot;
-  const int nA = (int)misc[2];
-  bool prod_ok = true;
+  const int nA = *s_na;
 
   if (warp == 0) {
-    // ------------------------------------------------ TMA producer (both CTAs)
+    // ------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t it = 0;
       int st = 0;
       uint32_t ph = 0;
-      const uint32_t full_cl = mapa_shared(smem_u32(full), 0);  // the even CTA's full[0]
-      auto load = [&](const ItemGeom& geo, int c0, int c1, int tp, int ot) -> bool {
-        for (int c = c0; c < c1; ++c) {
-          Chunk ch;
-          chunk_at(p, geo, s_tab, c, ch);
-          if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, p.st, 200 + st)) return false;
-          uint8_t* sb = smem + st * SB_STAGE;
-          const uint32_t fb = full_cl + 8u * (uint32_t)st;
-          const bool a = ch.which == 0;
-          if (rank == 0) mbar_arrive_expect_tx(&full[st], (a ? 4 : 3) * SB_BOX);  // both CTAs' boxes
-          tma_load_2d_pair(sb, &tm.x, fb, ch.xcol, (2 * tp + (int)rank) * SB_BM);
-          if (a)
-            tma_load_2d_pair(sb + SB_BOX, rank ? (const void*)&tm.e0 : (const void*)&tm.wb, fb, ch.bcol, ot * SB_BN);
-          else
-            tma_load_2d_pair(sb + SB_BOX, ch.which == 1 ? (const void*)&tm.dp : (const void*)&tm.dm, fb, ch.bcol,
-                             ot * SB_BN + (int)rank * (SB_BN / 2));
-          ++it;
-          if (++st == S) { st = 0; ph ^= 1; }
-        }
-        return true;
-      };
-      const ItemGeom geoA = item_geom(p, s_order, s_split, nA, 0);
-      int i = 0;
-      for (int u = cl; u < units && prod_ok; u += ncl, ++i) {
-        int tp, ot, tpn = 0, otn = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int tp, ot;
         unit_decode(p, u, tp, ot);
-        const bool nxt = MODE == kSbaAll && u + ncl < units;
-        if (nxt) unit_decode(p, u + ncl, tpn, otn);
-        if (MODE == kSbaPhaseA || (MODE == kSbaAll && i == 0)) prod_ok = load(geoA, 0, nA, tp, ot);
-        for (int s = 1; s < s_hi && prod_ok; ++s) {
-          const ItemGeom geo = item_geom(p, s_order, s_split, nA, s);
-          prod_ok = load(geo, 0, geo.nch, tp, ot);
-          if (prod_ok && nxt) prod_ok = load(geoA, pa_mark(nA, p.P, s - 1), pa_mark(nA, p.P, s), tpn, otn);
+        const int xrow0 = 2 * tp * SB_BM, xrow1 = xrow0 + SB_BM, brow = ot * SB_BN;
+        for (int step = s_lo; step < s_hi && ok; ++step) {
+          const ItemGeom geo = item_geom(p, s_order, s_split, nA, step);
+          const int nch = geo.nch;
+          for (int c = 0; c < nch; ++c) {
+            Chunk ch;
+            chunk_at(p, geo, s_tab, c, ch);
+            if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, p.st, 200 + st)) { ok = false; break; }
+            uint8_t* sb = smem + st * SB_STAGE;
+            mbar_arrive_expect_tx(&full[st], (ch.which == 0 ? 4 : 3) * SB_BOX);
+            tma_load_2d(sb, &tm.x, &full[st], ch.xcol, xrow0);
+            tma_load_2d(sb + SB_BOX, &tm.x, &full[st], ch.xcol, xrow1);
+            if (ch.which == 0) {
+              tma_load_2d(sb + 2 * SB_BOX, &tm.wb, &full[st], ch.bcol, brow);
+              tma_load_2d(sb + 3 * SB_BOX, &tm.e0, &full[st], ch.bcol, brow);
+            } else {
+              tma_load_2d(sb + 2 * SB_BOX, ch.which == 1 ? (const void*)&tm.dp : (const void*)&tm.dm, &full[st],
+                          ch.bcol, brow);
+            }
+            ++it;
+            if (++st == S) { st = 0; ph ^= 1; }
+          }
         }
-        if (prod_ok && nxt) prod_ok = load(geoA, pa_mark(nA, p.P, p.P - 1), nA, tpn, otn);
       }
-      // let every issued copy land before the CTA can exit: the even CTA's stage
-      // barriers count both CTAs' bytes (on a normal exit the MMAs have consumed
-      // every stage already)
-      if (rank == 0)
-        for (uint32_t j = (it > (uint32_t)S ? it - S : 0); j < it; ++j) mbar_drain(&full[j % S], (j / S) & 1);
-      else if (!prod_ok) {
-        const uint64_t t0 = global_ns();  // unwinding: give copies in flight time to land
-        while (global_ns() - t0 < 100000ull) {
-        }
-      }
+      // let every issued copy land before the CTA can exit
+      for (uint32_t j = (it > (uint32_t)S ? it - S : 0); j < it; ++j) mbar_drain(&full[j % S], (j / S) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------ MMA issuer (even CTA)
+    // ------------------------------------------------ MMA issuer
     // The issuing thread shares its SM sub-partition with four busy epilogue
     // warps, so its instruction stream per MMA is kept short: stage descriptors
     // come from one base by adding whole stages in 16-byte units, and the
     // 64-wide boxes' four K steps are unrolled.
-    if (lane == 0 && rank == 0) {
-      constexpr uint32_t idA = idesc_f16_f32(2 * SB_BM, 2 * SB_BN, false, false);  // phase A: y | d over the pair
-      constexpr uint32_t idS = idesc_f16_f32(2 * SB_BM, SB_BN, false, false);      // a step's update
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(SB_BM, SB_BN, false, false);
+      constexpr uint32_t idesc2 = idesc_f16_f32(SB_BM, 2 * SB_BN, false, false);
       constexpr uint64_t kStage16 = SB_STAGE / 16, kBox16 = SB_BOX / 16;
       const uint64_t d_first = sdesc_sw128(smem_u32(smem), 16, 1024);  // start-address field never carries (< 256 KB)
       uint64_t dcur = d_first;
       int st = 0;
-      uint32_t ph = 0;
+      uint32_t ph = 0, cnt = 0;
       bool ok = true;
+      const uint32_t ty0 = tbase, ty1 = tbase + 256;
       const bool dfull = p.g >= 64;  // delta chunks are whole 64-wide boxes
-      uint32_t nreg0 = 0u, nreg1 = 0u;  // units started per region
-      // wait until afree[R] has completed n phases (n = 0: a fresh region)
-      auto wait_free = [&](int R, uint32_t n) -> bool {
-        if (n == 0) return true;
-        return mbar_wait_cl(&afree[R], (n - 1) & 1, abort_flag, p.st, 220 + R);
-      };
-      // MMAs of one chunk (stage st) into accumulator columns dt
-      auto mma_chunk = [&](const ItemGeom& geo, int c, uint32_t dt) {
-        const uint64_t a0 = dcur, b0 = dcur + kBox16;
-        if (geo.step == 0) {
+      // The wait before a step's MMAs is for the epilogue's previous release of
+      // the slot; a unit's first step in kSbaSteps waits for the load of the
+      // unit's phase-A state instead, which is also the first completion of
+      // afree (in the other modes the first wait passes on the initial phase).
+      const uint32_t fpar = MODE == kSbaSteps ? 0u : 1u;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        for (int step = s_lo; step < s_hi && ok; ++step) {
+          if (!mbar_wait(&afree[0], (cnt & 1) ^ fpar, abort_flag, p.st, 220) ||
+              !mbar_wait(&afree[1], (cnt & 1) ^ fpar, abort_flag, p.st, 221)) { ok = false; break; }
+          tc_fence_after();
+          const ItemGeom geo = item_geom(p, s_order, s_split, nA, step);
+          const int nch = geo.nch;
+          // A shared-memory access by this thread while its MMAs are in flight
+          // waits for them to drain (about 380 cycles: the queue holds only a few
+          // MMAs), so each wait is made to cover two chunks where it can: right
+          // after the blocking wait on a chunk's stage, the next chunk of the
+          // same step is tested (cheap, nothing new in flight) and, if its stage
+          // is full too, both chunks go out behind the one wait. (Taking all
+          // three stages at once is slower: no stage is then being refilled
+          // while the MMAs run.)
+          for (int c = 0; c < nch;) {
+            if (!mbar_wait(&full[st], ph, abort_flag, p.st, 230 + st)) { ok = false; break; }
+            int st2 = st + 1;
+            uint32_t ph2 = ph;
+            if (st2 == S) { st2 = 0; ph2 ^= 1; }
+            const int take = (c + 1 < nch && mbar_test(&full[st2], ph2)) ? 2 : 1;
+            tc_fence_after();
+            for (int t = 0; t < take; ++t, ++c) {
+              const uint64_t a0 = dcur, a1 = dcur + kBox16, b0 = dcur + 2 * kBox16;
+              // advancing 32 bytes along K = +2 in the descriptor's 16-byte start-address field
+              if (step == 0) {
 #pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16)
-            tc_mma_f16_pair(dt, a0 + 2 * k16, b0 + 2 * k16, idA, (c > 0 || k16 > 0) ? 1u : 0u);
-        } else if (dfull) {
+                for (int k16 = 0; k16 < 4; ++k16) {
+                  const uint32_t acc = (c > 0 || k16 > 0) ? 1u : 0u;
+                  tc_mma_f16(ty0, a0 + 2 * k16, b0 + 2 * k16, idesc2, acc);
+                  tc_mma_f16(ty1, a1 + 2 * k16, b0 + 2 * k16, idesc2, acc);
+                }
+              } else if (dfull) {
+                // a step's update accumulates from zero (its own short chain); the
+                // epilogue adds it to d in registers
 #pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16)
-            tc_mma_f16_pair(dt, a0 + 2 * k16, b0 + 2 * k16, idS, (c > 0 || k16 > 0) ? 1u : 0u);
-        } else {
-          Chunk ch;
-          chunk_at(p, geo, s_tab, c, ch);
-          for (int k16 = ch.k16_lo; k16 < ch.k16_hi; ++k16)
-            tc_mma_f16_pair(dt, a0 + 2 * k16, b0 + 2 * k16, idS, (c > 0 || k16 > ch.k16_lo) ? 1u : 0u);
-        }
-        tc_commit_pair_mc(&empty[st], 3);
-        if (++st == S) { st = 0; ph ^= 1; dcur = d_first; } else { dcur += kStage16; }
-      };
-      // Chunks [c0, c1) of a step into accumulator columns dt, for phase A on
-      // its own (no candidate step to overlap): each wait is made to cover two
-      // chunks where it can (right after the blocking wait on a chunk's stage
-      // the next chunk's stage is tested, cheaply, nothing new being in flight).
-      auto issue = [&](const ItemGeom& geo, int c0, int c1, uint32_t dt) -> bool {
-        for (int c = c0; c < c1;) {
-          if (!mbar_wait(&full[st], ph, abort_flag, p.st, 230 + st)) return false;
-          int st2 = st + 1;
-          uint32_t ph2 = ph;
-          if (st2 == S) { st2 = 0; ph2 ^= 1; }
-          const int take = (c + 1 < c1 && mbar_test(&full[st2], ph2)) ? 2 : 1;
-          tc_fence_after();
-          for (int t = 0; t < take; ++t, ++c) mma_chunk(geo, c, dt);
-        }
-        return true;
-      };
-      const ItemGeom geoA = item_geom(p, s_order, s_split, nA, 0);
-      // Stages [st + t0, st + t1) of the ring (not consumed yet) filled.
-      auto prewait = [&](int t0, int t1) -> bool {
-        int st2 = st;
-        uint32_t ph2 = ph;
-        for (int t = 0; t < t1; ++t) {
-          if (t >= t0 && !mbar_wait(&full[st2], ph2, abort_flag, p.st, 230 + st2)) return false;
-          if (++st2 == S) { st2 = 0; ph2 ^= 1; }
-        }
-        return true;
-      };
-      // Chunks of candidate step s's period: the step, then the next unit's phase-A slice.
-      auto period_size = [&](int s, bool nxt) -> int {
-        const ItemGeom geo = item_geom(p, s_order, s_split, nA, s);
-        return geo.nch + (nxt ? pa_mark(nA, p.P, s) - pa_mark(nA, p.P, s - 1) : 0);
-      };
-      int i = 0;
-      for (int u = cl; u < units && ok; u += ncl, ++i) {
-        const int R = i & 1, Q = R ^ 1;
-        const uint32_t tR = tbase + 256u * R, tQ = tbase + 256u * Q;
-        const uint32_t base = (R ? nreg1 : nreg0) * Pl;  // afree[R] phases completed before this unit's
-        if (MODE == kSbaPhaseA || (MODE == kSbaAll && i == 0)) {
-          if (!wait_free(R, base)) break;
-          tc_fence_after();
-          if (!issue(geoA, 0, nA, tR)) break;
-          tc_commit_pair_mc(&afull[R], 3);
-        }
-        const bool nxt = MODE == kSbaAll && u + ncl < units;
-        if (nxt) {  // region Q free: the unit before this one is done with it
-          if (!wait_free(Q, (Q ? nreg1 : nreg0) * Pl)) break;
-          tc_fence_after();
-        }
-        // One period per candidate step: the step's chunks, then a slice of the
-        // next unit's phase A. A wait by this thread behind MMAs in flight holds
-        // it until they drain, so each period has one such wait: the next
-        // period's stages are waited for right after this period's MMAs go out
-        // (the epilogue is reading and computing meanwhile), the accumulator's
-        // release then with nothing in flight, and the period's MMAs follow
-        // back to back.
-        int pw = 0;  // stages of the coming period already waited for
-        for (int s = 1; s < s_hi; ++s) {
-          const ItemGeom geo = item_geom(p, s_order, s_split, nA, s);
-          const int a0 = nxt ? pa_mark(nA, p.P, s - 1) : 0, a1 = nxt ? pa_mark(nA, p.P, s) : 0;
-          const int ns = geo.nch, total = ns + (a1 - a0);
-          const int pre = total < S ? total : S;
-          if (pw < pre && !prewait(pw, pre)) { ok = false; break; }
-          if (!wait_free(R, base + (uint32_t)s)) { ok = false; break; }
-          tc_fence_after();
-          for (int t = 0; t < total; ++t) {
-            if (t >= pre) {
-              if (!mbar_wait(&full[st], ph, abort_flag, p.st, 230 + st)) { ok = false; break; }
-              tc_fence_after();
-            }
-            if (t < ns) {
-              mma_chunk(geo, t, tR + SB_BN);
-              if (t == ns - 1) tc_commit_pair_mc(&afull[R], 3);
-            } else {
-              mma_chunk(geoA, a0 + (t - ns), tQ);
+                for (int k16 = 0; k16 < 4; ++k16) {
+                  const uint32_t acc = (c > 0 || k16 > 0) ? 1u : 0u;
+                  tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, acc);
+                  tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, acc);
+                }
+              } else {
+                Chunk ch;
+                chunk_at(p, geo, s_tab, c, ch);
+                for (int k16 = ch.k16_lo; k16 < ch.k16_hi; ++k16) {
+                  const uint32_t acc = (c > 0 || k16 > ch.k16_lo) ? 1u : 0u;
+                  tc_mma_f16(ty0 + 128, a0 + 2 * k16, b0 + 2 * k16, idesc, acc);
+                  tc_mma_f16(ty1 + 128, a1 + 2 * k16, b0 + 2 * k16, idesc, acc);
+                }
+              }
+              tc_commit(&empty[st]);
+              if (++st == S) { st = 0; ph ^= 1; dcur = d_first; } else { dcur += kStage16; }
             }
           }
           if (!ok) break;
-          pw = 0;
-          if (s + 1 < s_hi) {
-            const int t2 = period_size(s + 1, nxt);
-            pw = t2 < S ? t2 : S;
-            if (!prewait(0, pw)) { ok = false; break; }
-          }
+          tc_commit(&afull[0]);
+          tc_commit(&afull[1]);
+          ++cnt;
         }
-        if (!ok) break;
-        if (nxt) {
-          if (!issue(geoA, pa_mark(nA, p.P, p.P - 1), nA, tQ)) break;
-          tc_commit_pair_mc(&afull[Q], 3);
-        }
-        if (R) ++nreg1; else ++nreg0;
       }
-      tc_commit_pair(done);
+      tc_commit(done);
       mbar_drain(done, 0);
     }
   } else {
-    // ------------------------------------------------ epilogue (both CTAs)
-    // warp e = warp - 2: TMEM lane quadrant q = warp & 3 (the quadrant a warp
-    // may access), column quarter h = e >> 2; row r = 32 q + lane.
+    // ------------------------------------------------ epilogue
+    // warp e = warp - 2: slot e >> 3, column half h = (e >> 2) & 1, TMEM lane
+    // quadrant q = warp & 3 (the quadrant a warp may access); row r = 32 q + lane.
     const int e = warp - 2;
-    const int q = warp & 3, h = e >> 2;
+    const int slot = e >> 3, h = (e >> 2) & 1, q = warp & 3;
     const int r = q * 32 + lane;
     const int F = 2 + 2 * p.P;
-    const uint32_t afree_cl = mapa_shared(smem_u32(afree), 0);
-    uint32_t ecnt0 = 0u, ecnt1 = 0u, scnt = 0;  // afull phases consumed per region; sums exchanges
+    const uint32_t ty = tbase + ((uint32_t)(q * 32) << 16) + slot * 256 + h * 64, td = ty + 128;
+    float* xs = s_x + (slot * 128 + r) * 12;  // [0..3] even steps, [4..7] odd steps, [8..9] shifts
+    uint64_t* xb = xbar + (slot * 4 + q) * 4;  // max h0, max h1, sums (even), sums (odd)
+    uint32_t cnt = 0, nunit = 0;
     bool ok = true;
-    auto release = [&](int R) {
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(afree_cl + 8u * (uint32_t)R);
-    };
-    int i = 0;
-    for (int u = cl; u < units && ok; u += ncl, ++i) {
-      const int R = i & 1;
-      const uint32_t ty = tbase + ((uint32_t)(q * 32) << 16) + 256u * R + 32u * h, td = ty + SB_BN;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++nunit) {
       int tp, ot;
       unit_decode(p, u, tp, ot);
-      const int tt = 2 * tp + (int)rank;
-      const bool have = tt < p.n_tt;  // the second tile of an odd pair is padding
-      const int64_t col0 = (int64_t)ot * SB_BN + 32 * h;
-      const int nvalid = (int)((p.m - col0) > 32 ? 32 : ((p.m - col0) > 0 ? (p.m - col0) : 0));
+      const int tt = 2 * tp + slot;
+      const bool have = tt < p.n_tt;        // the second tile of an odd pair is padding
+      const int64_t col0 = (int64_t)ot * SB_BN + h * 64;
+      const int nvalid = (int)((p.m - col0) > 64 ? 64 : ((p.m - col0) > 0 ? (p.m - col0) : 0));
       float* outp = p.part + ((size_t)(have ? tt : 0) * p.n_ot + ot) * F * SB_BM + r;
-      // this thread's 32 outputs of its token row in yd (e^(y - M); d at + 128 rows)
-      float* ydp = p.yd + ((size_t)(have ? tt : 0) * p.n_ot + ot) * 2 * SB_BN * SB_BM + (size_t)(32 * h) * SB_BM + r;
+      // this thread's 64 outputs of its token row in yd (e^(y - M); d at + 128 rows)
+      float* ydp = p.yd + ((size_t)(have ? tt : 0) * p.n_ot + ot) * 2 * SB_BN * SB_BM + (size_t)(h * 64) * SB_BM + r;
       float Mt = 0.f;
-      uint32_t ecnt = R ? ecnt1 : ecnt0;
-      // d of this thread's 32 outputs, kept in registers for the whole unit: phase A
+      // d of this thread's 64 outputs, kept in registers for the whole unit: phase A
       // leaves d_0 in tensor memory, every later step its update alone, added here
       // with round-to-nearest fp32 adds (the tensor core's accumulator truncates,
       // which over the long chain of all steps would shrink |d| systematically)
-      uint32_t v[32];
+      uint32_t v[64];
       if (MODE == kSbaSteps) {
         // phase A's e^(y - M) back in tensor memory and its d_0 into registers; the
-        // arrival hands the region to the first candidate step's MMAs
-        uint32_t t[32];
+        // arrival on afree hands the slot to the first candidate step's MMAs (a
+        // unit's last step does not release the slot in this mode: this load does)
 #pragma unroll
-        for (int j = 0; j < 32; ++j) t[j] = have ? __float_as_uint(ydp[(size_t)j * SB_BM]) : 0u;
-        tmem_st32(ty, t);
+        for (int j = 0; j < 64; ++j) v[j] = have ? __float_as_uint(ydp[(size_t)j * SB_BM]) : 0u;
+        tmem_st32(ty, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_st32(ty + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tc_wait_st();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = have ? __float_as_uint(ydp[(size_t)(SB_BN + j) * SB_BM]) : 0u;
-        release(R);
+        for (int j = 0; j < 64; ++j) v[j] = have ? __float_as_uint(ydp[(size_t)(SB_BN + j) * SB_BM]) : 0u;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afree[slot]);
       }
-      // The tail of every step: the sums of this step's d over the thread's 32
-      // outputs (ev: their e^(y - M); dm: the largest d), and the quarters'
-      // exchange and partial stores. false: a wait gave up.
-      auto finish_step = [&](int step, float sy, const uint32_t (&ev)[32], float dm) -> bool {
-        // Per-token sums over this thread's 32 outputs. KL: S_q = sum e^(y-M) e^d
+      // The tail of every step: the sums of this step's d over the thread's 64
+      // outputs, the accumulator's release after the unit's last step, and the
+      // halves' exchange and partial stores. false: a wait gave up.
+      auto finish_step = [&](int step, float sy) -> bool {
+        const bool last = step == s_hi - 1;
+        // Per-token sums over this thread's 64 outputs. KL: S_q = sum e^(y-M) e^d
         // and A = sum e^(y-M) d. MSE: the sum of d^2 (accumulator units, x 2^16).
         uint64_t sqp = 0, ap = 0;  // packed (even, odd column) sums
         float csh = 0.f;           // S_q carries a factor 2^-csh (0 unless it could overflow)
         if (OBJ == 1) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
+          for (int j = 0; j < 64; j += 2) {
             const uint64_t dd = f2_pack(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
             sqp = f2_fma(dd, dd, sqp);
           }
@@ -708,160 +610,169 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           // exponent decides a shift csh, a multiple of 32 that keeps every term
           // at most 2^64; it is 0 for ordinary layers, where e^(d log2(e) - 0)
           // is exactly the unshifted term.
+          float dm = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+#pragma unroll
+          for (int j = 3; j < 63; j += 2) dm = fmax3(dm, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+          dm = fmaxf(dm, __uint_as_float(v[63]));
           const float c = dm * kC1 - 64.f;
           csh = c > 0.f ? 32.f * ceilf(c * (1.f / 32.f)) : 0.f;
           const uint64_t kc2 = f2_pack(kC1, kC1), nc = f2_pack(-csh, -csh);
+          // e^(y - M) in 8-column pieces. In the split launches the pieces are
+          // double-buffered (the load of the next one is in flight while this one
+          // is consumed); the one-pass launch loads them one at a time. Same
+          // arithmetic either way.
+          constexpr int NB = MODE == kSbaAll ? 1 : 2;
+          uint32_t ev[NB][8];
+          if (NB == 2) {
+            tmem_ld8(ty, ev[0]);
+            tc_wait_ld8(ev[0]);
+          }
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const uint64_t ey = f2_pack(__uint_as_float(ev[j]), __uint_as_float(ev[j + 1]));
-            const uint64_t dd = f2_pack(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-            float x0, x1;
-            f2_unpack(f2_fma(dd, kc2, nc), x0, x1);
-            sqp = f2_fma(ey, f2_pack(ex2(x0), ex2(x1)), sqp);
-            ap = f2_fma(ey, dd, ap);
+          for (int cc = 0; cc < 8; ++cc) {
+            uint32_t (&cur)[8] = ev[cc % NB];
+            if (NB == 1) {
+              tmem_ld8(ty + cc * 8, cur);
+              tc_wait_ld8(cur);
+            } else if (cc + 1 < 8) {
+              tmem_ld8(ty + (cc + 1) * 8, ev[(cc + 1) % NB]);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+              const uint64_t ey = f2_pack(__uint_as_float(cur[j]), __uint_as_float(cur[j + 1]));
+              const uint64_t dd = f2_pack(__uint_as_float(v[cc * 8 + j]), __uint_as_float(v[cc * 8 + j + 1]));
+              float x0, x1;
+              f2_unpack(f2_fma(dd, kc2, nc), x0, x1);
+              sqp = f2_fma(ey, f2_pack(ex2(x0), ex2(x1)), sqp);
+              ap = f2_fma(ey, dd, ap);
+            }
+            if (NB == 2 && cc + 1 < 8) tc_wait_ld8(ev[(cc + 1) % NB]);
           }
         }
         float sq0, sq1, a0, a1;
         f2_unpack(sqp, sq0, sq1);
         f2_unpack(ap, a0, a1);
-        // quarters 1..3 hand their sums to quarter 0, which writes the row's partials
-        const int par = scnt & 1;
-        if (h != 0) {
-          float* xo = s_x + (8 + (par * 3 + h - 1) * 4) * SB_BM + r;
-          xo[0] = sy;
-          xo[SB_BM] = sq0 + sq1;
-          xo[2 * SB_BM] = a0 + a1;
-          xo[3 * SB_BM] = csh;
+        if (last && MODE != kSbaSteps) {
+          tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&xbs[q * 2 + par]);
+          if (lane == 0) mbar_arrive(&afree[slot]);
+        }
+        // half 1 hands its sums to half 0, which writes the row's partials
+        const int par = cnt & 1;
+        float* xo = xs + 4 * par;
+        if (h == 1) {
+          xo[1] = sy;
+          xo[2] = sq0 + sq1;
+          xo[3] = a0 + a1;
+          xs[8 + par] = csh;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&xb[2 + par]);
         } else {
-          if (!mbar_wait(&xbs[q * 2 + par], (scnt >> 1) & 1, abort_flag, p.st, 252)) return false;
+          if (!mbar_wait(&xb[2 + par], (cnt >> 1) & 1, abort_flag, p.st, 252 + slot)) return false;
           if (have) {
-            const float* xi = s_x + (8 + par * 3 * 4) * SB_BM + r;
-            float syt = sy, sq = sq0 + sq1, at = a0 + a1, ct = csh;
-            bool shifted = csh != 0.f;
-#pragma unroll
-            for (int hh = 0; hh < 3; ++hh) {
-              syt += xi[(4 * hh) * SB_BM];
-              sq += xi[(4 * hh + 1) * SB_BM];
-              at += xi[(4 * hh + 2) * SB_BM];
-              const float c2 = xi[(4 * hh + 3) * SB_BM];
-              shifted |= c2 != 0.f;
-              ct = fmaxf(ct, c2);
-            }
             if (step == 0) {
               outp[0] = Mt * kOpUnscale;
-              outp[SB_BM] = syt;
+              outp[SB_BM] = sy + xo[1];
             }
-            // S_q of the row: the plain sum when no quarter is shifted (the usual
-            // case); else the quarters at a common shift, stored as the value if
-            // it fits below 2^120 and otherwise as minus its log2 (S_q > 0, so a
-            // negative entry is unambiguous)
-            if (shifted) {
-              float s2 = pow2i(csh - ct) * (sq0 + sq1);
-#pragma unroll
-              for (int hh = 0; hh < 3; ++hh)
-                s2 += pow2i(xi[(4 * hh + 3) * SB_BM] - ct) * xi[(4 * hh + 1) * SB_BM];
+            // S_q of the row: the plain sum when neither half is shifted (the
+            // usual case); else the halves at a common shift, stored as the
+            // value if it fits below 2^120 and otherwise as minus its log2
+            // (S_q > 0, so a negative entry is unambiguous)
+            const float c1 = xs[8 + par];
+            float sq = (sq0 + sq1) + xo[2];
+            if (csh != 0.f || c1 != 0.f) {
+              const float ct = fmaxf(csh, c1);
+              const float s2 = pow2i(csh - ct) * (sq0 + sq1) + pow2i(c1 - ct) * xo[2];
               const float l2 = log2f(s2) + ct;
               sq = l2 < 120.f ? exp2f(l2) : -l2;
             }
             outp[(size_t)(2 + 2 * step) * SB_BM] = sq;
-            outp[(size_t)(3 + 2 * step) * SB_BM] = at * kOpUnscale;
+            outp[(size_t)(3 + 2 * step) * SB_BM] = ((a0 + a1) + xo[3]) * kOpUnscale;
           }
         }
-        ++scnt;
+        ++cnt;
         return true;
       };
-      // After the reads of each step, the region goes back to the MMA issuer: as
-      // the next step's accumulator, or (after the unit's last step, when e^(y - M)
-      // has been read too) for the unit after next.
+      // the accumulator's release once its contents are in registers (not after
+      // the unit's last step: the next unit's first MMA overwrites e^(y - M))
+      auto release_early = [&](int step) {
+        if (step != s_hi - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afree[slot]);
+        }
+      };
       if (MODE != kSbaSteps) {
-        // step 0 (phase A): y -> row maximum (all four quarters) -> e^(y - M)
-        // stored back in place of y; then d_0 into registers
-        if (!mbar_wait(&afull[R], ecnt & 1, abort_flag, p.st, 240 + R, p.acc_wait_ns)) { ok = false; break; }
-        ++ecnt;
+        // step 0 (phase A): y -> row maximum (both halves) -> e^(y - M) stored back
+        // in place of y; then d_0 into registers
+        if (!mbar_wait(&afull[slot], cnt & 1, abort_flag, p.st, 240 + slot, p.acc_wait_ns)) { ok = false; break; }
         tc_fence_after();
-        uint32_t yv[32];
-        tmem_ld32(ty, yv);
-        tc_wait_ld32(yv);
+        // y in 8-column pieces (the maximum, then e^(y - M) written back in
+        // place), so that no 64 registers besides d are needed
+        float sy = 0.f;
         float mx = -3.0e38f;
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nvalid) mx = fmaxf(mx, __uint_as_float(yv[j]));
-        float* xm = s_x + ((i & 1) * 4) * SB_BM + r;  // this unit's maximum slots (double-buffered)
-        xm[h * SB_BM] = mx;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&xbm[q]);
-        if (!mbar_wait(&xbm[q], i & 1, abort_flag, p.st, 250 + q)) { ok = false; break; }
-        mx = fmaxf(fmaxf(xm[0], xm[SB_BM]), fmaxf(xm[2 * SB_BM], xm[3 * SB_BM]));
-        const float mb = -mx * kC1;
-        float sy = 0.f;
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t yv[8];
+          tmem_ld8(ty + cc * 8, yv);
+          tc_wait_ld8(yv);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float ey = (j < nvalid) ? ex2(fmaf(__uint_as_float(yv[j]), kC1, mb)) : 0.f;
-          sy += ey;
-          yv[j] = __float_as_uint(ey);
-          if (MODE == kSbaPhaseA && have) ydp[(size_t)j * SB_BM] = ey;
+          for (int j = 0; j < 8; ++j)
+            if (cc * 8 + j < nvalid) mx = fmaxf(mx, __uint_as_float(yv[j]));
         }
-        tmem_st32(ty, yv);
+        xs[h ? 0 : 4] = mx;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xb[h]);
+        if (!mbar_wait(&xb[h ^ 1], nunit & 1, abort_flag, p.st, 250 + slot)) { ok = false; break; }
+        mx = fmaxf(mx, xs[h ? 4 : 0]);
+        const float mb = -mx * kC1;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t yv[8];
+          tmem_ld8(ty + cc * 8, yv);
+          tc_wait_ld8(yv);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float ey = (cc * 8 + j < nvalid) ? ex2(fmaf(__uint_as_float(yv[j]), kC1, mb)) : 0.f;
+            sy += ey;
+            yv[j] = __float_as_uint(ey);
+            if (MODE == kSbaPhaseA && have) ydp[(size_t)(cc * 8 + j) * SB_BM] = ey;
+          }
+          tmem_st8(ty + cc * 8, yv);
+        }
         tc_wait_st();
         Mt = mx;
-        tmem_ld32(td, v);
-        tc_wait_ld32(v);
+        tmem_ld32(td, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(td + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tc_wait_ld();
         if (MODE == kSbaPhaseA && have) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) ydp[(size_t)(SB_BN + j) * SB_BM] = __uint_as_float(v[j]);
+          for (int j = 0; j < 64; ++j) ydp[(size_t)(SB_BN + j) * SB_BM] = __uint_as_float(v[j]);
         }
-        release(R);
-        float dm = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
-#pragma unroll
-        for (int j = 3; j < 31; j += 2) dm = fmax3(dm, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-        dm = fmaxf(dm, __uint_as_float(v[31]));
-        if (!finish_step(0, sy, yv, dm)) { ok = false; break; }
+        release_early(0);
+        if (!finish_step(0, sy)) { ok = false; break; }
       }
       for (int step = 1; step < s_hi; ++step) {
-        // candidate step: e^(y - M) read ahead of the accumulator's wait; then
-        // d += this step's update (round to nearest), its largest entry on the way
-        uint32_t ev[32];
-        if (OBJ == 0) {
-          tmem_ld16(ty, *reinterpret_cast<uint32_t(*)[16]>(&ev[0]));
-          tmem_ld16(ty + 16, *reinterpret_cast<uint32_t(*)[16]>(&ev[16]));
-        }
-        if (!mbar_wait(&afull[R], ecnt & 1, abort_flag, p.st, 240 + R, p.acc_wait_ns)) { ok = false; break; }
-        ++ecnt;
+        // candidate step: d += this step's update (round to nearest)
+        if (!mbar_wait(&afull[slot], cnt & 1, abort_flag, p.st, 240 + slot, p.acc_wait_ns)) { ok = false; break; }
         tc_fence_after();
-        float dm = -3.0e38f;
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          uint32_t a8[8];
-          tmem_ld8(td + 8 * qq, a8);
-          tc_wait_ld8(a8);
+        for (int q = 0; q < 4; ++q) {
+          uint32_t u[16];
+          tmem_ld16(td + 16 * q, u);
+          tc_wait_ld16(u);
 #pragma unroll
-          for (int j = 0; j < 8; j += 2) {
-            float x0, x1;
-            f2_unpack(f2_add(f2_pack(__uint_as_float(v[8 * qq + j]), __uint_as_float(v[8 * qq + j + 1])),
-                             f2_pack(__uint_as_float(a8[j]), __uint_as_float(a8[j + 1]))),
-                      x0, x1);
-            v[8 * qq + j] = __float_as_uint(x0);
-            v[8 * qq + j + 1] = __float_as_uint(x1);
-            dm = fmax3(dm, x0, x1);
-          }
+          for (int j = 0; j < 16; ++j)
+            v[16 * q + j] = __float_as_uint(__fadd_rn(__uint_as_float(v[16 * q + j]), __uint_as_float(u[j])));
         }
-        if (OBJ == 0) tc_wait_ld32(ev);  // (already complete: names ev for the compiler)
-        release(R);
-        if (!finish_step(step, 0.f, ev, dm)) { ok = false; break; }
+        release_early(step);
+        if (!finish_step(step, 0.f)) { ok = false; break; }
       }
-      if (R) ecnt1 = ecnt; else ecnt0 = ecnt;
     }
   }
-  (void)prod_ok;
-  // the peer's barriers and shared memory stay in use until both CTAs are done
-  tc_fence_before();
-  cluster_sync_all();
+  __syncthreads();
   if (warp == 1) {
-    __syncwarp();
     tc_fence_after();
-    tmem_dealloc_pair(tbase, 512);
+    tmem_dealloc(tbase, 512);
   }
 }
 
@@ -1036,9 +947,9 @@ SbaPlan sba_plan(int64_t m, int64_t n, int64_t N, int xdtype, int group) {
   }
   pl.off_klp = off; off = align256(off + (size_t)pl.P * pl.n_tt * sizeof(double));
   pl.total = off;
-  const size_t fixed = 1024 + (size_t)(2 * SB_MAX_STAGES + 17) * 8 + 16 + (size_t)((pl.k + 3) & ~3) * 4 +
-                       (size_t)SB_XF * SB_BM * sizeof(float) + (size_t)3 * pl.nbox * 2 + (size_t)pl.nbox + 64;
-  int st = SB_MAX_STAGES;
+  const size_t fixed = 1024 + 512 + 256 + (size_t)(pl.k + 4) * 4 + 64 + 2 * 128 * 12 * sizeof(float) +
+                       (size_t)3 * pl.nbox * 2 + (size_t)((pl.nbox + 15) & ~15) + 16;
+  int st = 3;
   while (st > 2 && fixed + (size_t)st * SB_STAGE > 227 * 1024) --st;
   pl.stages = st;
   pl.smem = fixed + (size_t)st * SB_STAGE;
@@ -1230,8 +1141,8 @@ static cudaError_t launch_score(const SbaPlan& pl, int64_t m, int64_t n, int64_t
   const uint64_t wcols = 2 * (uint64_t)pl.npad;  // hi | lo
   ok = ok && make_tmap_f16(&tm.wb, pw + pl.off_wb, wcols, (uint64_t)m, SB_BK, SB_BN);
   ok = ok && make_tmap_f16(&tm.e0, pw + pl.off_e0, wcols, (uint64_t)m, SB_BK, SB_BN);
-  ok = ok && make_tmap_f16(&tm.dp, pw + pl.off_dp, wcols, (uint64_t)m, SB_BK, SB_BN / 2);
-  ok = ok && make_tmap_f16(&tm.dm, pw + pl.off_dm, wcols, (uint64_t)m, SB_BK, SB_BN / 2);
+  ok = ok && make_tmap_f16(&tm.dp, pw + pl.off_dp, wcols, (uint64_t)m, SB_BK, SB_BN);
+  ok = ok && make_tmap_f16(&tm.dm, pw + pl.off_dm, wcols, (uint64_t)m, SB_BK, SB_BN);
   if (!ok) return cudaErrorInvalidValue;
   SbaParams p;
   p.N = N; p.m = m; p.n = n; p.npad = pl.npad; p.g = group; p.k = pl.k; p.P = pl.P; p.ksplit = pl.ksplit;
@@ -1246,48 +1157,23 @@ static cudaError_t launch_score(const SbaPlan& pl, int64_t m, int64_t n, int64_t
     const unsigned long long v = std::strtoull(t, nullptr, 10);
     if (v > 0 && v < kWaitLimitNs) p.acc_wait_ns = v;
   }
-  auto kern = objective == 1 ? sba_score_kernel<MODE, 1> : sba_score_kernel<MODE, 0>;
   static std::atomic<uint64_t> attr{0};
-  static int max_pairs[64];
   uint64_t bit = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
   if (attr_pending(attr, bit)) {  // the plan's shared memory never exceeds this bound
-    for (auto f : {sba_score_kernel<MODE, 0>, sba_score_kernel<MODE, 1>}) {
-      cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-      if (e != cudaSuccess) return e;
-    }
-    max_pairs[dev & 63] = 0;
+    cudaError_t e = cudaFuncSetAttribute(sba_score_kernel<MODE, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         227 * 1024);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(sba_score_kernel<MODE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
     attr.fetch_or(bit);
   }
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute cattr[1];
-  cattr[0].id = cudaLaunchAttributeClusterDimension;
-  cattr[0].val.clusterDim.x = 2;
-  cattr[0].val.clusterDim.y = 1;
-  cattr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(SB_THREADS);
-  cfg.dynamicSmemBytes = pl.smem;
-  cfg.stream = s;
-  cfg.attrs = cattr;
-  cfg.numAttrs = 1;
-  // CTA pairs that fit on the device at once (one CTA per SM; the GPC layout can
-  // leave an SM without a partner)
-  if (max_pairs[dev & 63] <= 0) {
-    int nc = 0;
-    cfg.gridDim = dim3((unsigned)(num_sms & ~1));
-    if (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) != cudaSuccess || nc <= 0) {
-      cudaGetLastError();
-      nc = num_sms / 2;
-    }
-    max_pairs[dev & 63] = nc;
-  }
   const int units = p.n_tp * pl.n_ot;
-  const int pairs = units < max_pairs[dev & 63] ? units : max_pairs[dev & 63];
-  cfg.gridDim = dim3((unsigned)(2 * pairs));
+  const int grid = units < num_sms ? units : num_sms;
   if (kev) cudaEventRecord(kev[0], s);
-  cudaError_t le = cudaLaunchKernelEx(&cfg, kern, tm, p);
-  if (le != cudaSuccess) return le;
+  if (objective == 1)
+    sba_score_kernel<MODE, 1><<<grid, SB_THREADS, pl.smem, s>>>(tm, p);
+  else
+    sba_score_kernel<MODE, 0><<<grid, SB_THREADS, pl.smem, s>>>(tm, p);
   if (kev) cudaEventRecord(kev[1], s);
   count_launches(1);
   return cudaGetLastError();
