@@ -333,7 +333,7 @@ def extra_kernels(spec, Wd, Xd, d, stages, flush, stream):
     for B in (1, 8):
         x = torch.randn((B, n), device=Wd.device).to(torch.bfloat16)
         ys = [torch.empty((B, m), dtype=torch.float32, device=Wd.device) for _ in range(ncopy)]
-        gws = torch.empty(slim._lib().slim_dequant_gemv_workspace_bytes(m, n, spec.group, B), dtype=torch.uint8,
+        gws = torch.empty(max(256, slim._lib().slim_dequant_gemv_workspace_bytes(m, n, spec.group, spec.avg_bits, B)), dtype=torch.uint8,
                           device=Wd.device)
         side = torch.cuda.Stream(device=Wd.device)
         side.wait_stream(stream)

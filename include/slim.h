@@ -303,10 +303,11 @@ int slim_gptq(const float* W, int64_t m, int64_t n, const double* H, const uint8
  * batch is 1..8. Arithmetic: fp32 (each code times x in one fma). The call is
  * asynchronous: it returns once the kernels are enqueued on `stream` (host-side
  * argument checks only), so decode loops can issue it back to back. Workspace:
- * slim_dequant_gemv_workspace_bytes; ws NULL takes it from the library's pool
- * and returns it in stream order.
+ * slim_dequant_gemv_workspace_bytes (0 when one launch covers every group of a
+ * row, as for the usual layer shapes); ws NULL takes it from the library's
+ * pool and returns it in stream order.
  */
-size_t slim_dequant_gemv_workspace_bytes(int64_t m, int64_t n, int group, int64_t batch);
+size_t slim_dequant_gemv_workspace_bytes(int64_t m, int64_t n, int group, int avg_bits, int64_t batch);
 int slim_dequant_gemv(const uint32_t* codes, const uint8_t* bits, const float* scale, const float* zero,
                       int64_t m, int64_t n, int group, int avg_bits, const void* x, int xdtype,
                       int64_t batch, float* y, void* ws, size_t ws_bytes, void* stream);

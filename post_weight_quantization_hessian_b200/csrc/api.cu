@@ -54,10 +54,10 @@ cudaError_t launch_sba_select(const float* W, const void* X, int64_t m, int64_t 
                               int precision, uint8_t* pw, uint8_t* sw, cudaStream_t s);
 cudaError_t launch_order_check(const int32_t* order, int k, int32_t* out, DevStatus* st, cudaStream_t s);
 size_t gptq_workspace_doubles(int64_t m, int64_t n);
-size_t dg_workspace_bytes(int64_t m, int64_t n, int group, int64_t B, int num_sms);
+size_t dg_workspace_bytes(int64_t m, int64_t n, int group, int avg_bits, int64_t B);
 cudaError_t launch_dequant_gemv(const uint32_t* codes, const uint8_t* bits, const float* scale, const float* zero,
                                 int64_t m, int64_t n, int group, int avg_bits, const void* x, int xdtype, int B,
-                                float* y, uint8_t* ws, int num_sms, cudaStream_t s);
+                                float* y, uint8_t* ws, cudaStream_t s);
 cudaError_t launch_gptq(const float* W, int64_t m, int64_t n, const double* H, double alpha, const uint8_t* bits,
                         int group, int avg_bits, double lam, int n_tau, uint32_t* codes, float* scale, float* zero,
                         uint8_t* tau_idx, double* h, double* ws, DevStatus* st, int num_sms, cudaStream_t s);
@@ -181,6 +181,10 @@ struct Workspace {
     if (ws) {
       if (ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255)) return SLIM_EINVAL;
       p = static_cast<uint8_t*>(ws);
+      return SLIM_OK;
+    }
+    if (need == 0) {  // nothing to allocate
+      p = nullptr;
       return SLIM_OK;
     }
     cudaMemPool_t pool;
@@ -539,11 +543,9 @@ int slim_gptq(const float* W, int64_t m, int64_t n, const double* H, const uint8
 }
 
 // ------------------------------------------------------------------ dequant gemv
-size_t slim_dequant_gemv_workspace_bytes(int64_t m, int64_t n, int group, int64_t batch) {
-  int sms = 0;
-  if (device_sms(&sms) != SLIM_OK) sms = 148;
-  if (m < 1 || n < 1 || group < 32 || n % group || batch < 1) return 0;
-  return al256(dg_workspace_bytes(m, n, group, batch, sms));
+size_t slim_dequant_gemv_workspace_bytes(int64_t m, int64_t n, int group, int avg_bits, int64_t batch) {
+  if (m < 1 || n < 1 || group < 32 || n % group || batch < 1 || batch > 8 || avg_bits < 1 || avg_bits > 8) return 0;
+  return al256(dg_workspace_bytes(m, n, group, avg_bits, batch));
 }
 
 int slim_dequant_gemv(const uint32_t* codes, const uint8_t* bits, const float* scale, const float* zero, int64_t m,
@@ -555,7 +557,6 @@ int slim_dequant_gemv(const uint32_t* codes, const uint8_t* bits, const float* s
   rc = check_bits(avg_bits);
   if (rc) return rc;
   if (batch < 1 || batch > 8 || (n * avg_bits) % 32) return SLIM_EINVAL;
-  if ((m + 31) / 32 > (int64_t)65535 * 4) return SLIM_EINVAL;
   int sms = 0;
   rc = device_sms(&sms);
   if (rc) return rc;
@@ -563,10 +564,9 @@ int slim_dequant_gemv(const uint32_t* codes, const uint8_t* bits, const float* s
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Workspace w;
   w.sync_on_release = false;
-  rc = w.acquire(ws, ws_bytes, slim_dequant_gemv_workspace_bytes(m, n, group, batch), s);
+  rc = w.acquire(ws, ws_bytes, slim_dequant_gemv_workspace_bytes(m, n, group, avg_bits, batch), s);
   if (rc) return rc;
-  SLIM_CUDA(launch_dequant_gemv(codes, bits, scale, zero, m, n, group, avg_bits, x, xdtype, (int)batch, y, w.p, sms,
-                                s));
+  SLIM_CUDA(launch_dequant_gemv(codes, bits, scale, zero, m, n, group, avg_bits, x, xdtype, (int)batch, y, w.p, s));
   return SLIM_OK;
 }
 

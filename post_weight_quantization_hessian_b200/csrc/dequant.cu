@@ -13,51 +13,74 @@
 // batch row, shared by all rows). Per code that is a funnel shift, one
 // logical op and one fma.
 //
-// Layout of the work: lane = output row (32 rows per warp), so every lane of a
-// warp decodes the same code positions (uniform control flow, x read by all
-// lanes at one address); each lane reads its own row's words of a group
-// (whole groups are whole words). The groups are split over gridDim.y warps
-// per row block, so that enough loads are in flight; their partial sums go to
-// a fixed-order reduction (deterministic). Batch rows: up to 8, each code's f
-// reused for all of them. HBM-bound on the codes and the per-group scale and
-// zero at batch 1.
+// Layout of the work. A block takes 32 output rows and a range of groups
+// (all of them unless a row's words would not fit in shared memory). It first
+// copies the rows' packed words, scales and zeros into shared memory with
+// coalesced asynchronous copies (consecutive threads take consecutive words of
+// one row, all in flight at once; the rows are stored at an odd word stride),
+// and sums x over each group of the range; then each of its 8 warps decodes every 8th group with lane = row, so
+// that all lanes decode the same code positions (uniform control flow, one x
+// address per warp) and read their own row's words from shared memory without
+// bank conflicts. The warps' sums are added in a fixed order: one launch, no
+// atomics, deterministic. Batch rows: up to 8, each code's f reused for all of
+// them. HBM-bound on the codes, scales and zeros at batch 1.
+#include <algorithm>
 #include <cstdint>
 #include "common.cuh"
 
 namespace slim {
 
-constexpr int DG_WARPS = 4;
-constexpr int DG_MAXB = 8;
+constexpr int DG_WARPS = 8;
+constexpr int DG_ROWS = 32;
+constexpr size_t DG_SMEM_MAX = 100 * 1024;  // two blocks per SM
 
-// One warp per (batch row b, group c): x of the group's G columns as fp32
-// (bf16 widened exactly) into xf, their sum into xs[b][c].
-__global__ void dg_prep_kernel(int k, int G, const void* __restrict__ x, int xdtype, int B, int64_t n,
-                               float* __restrict__ xf, float* __restrict__ xs) {
-  const int lane = threadIdx.x & 31;
-  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (e >= B * k) return;
-  const int b = e / k, c = e - b * k;
-  const int64_t base = (int64_t)b * n + (int64_t)c * G;
-  float s = 0.f;
-  for (int j = lane; j < G; j += 32) {
-    float v;
-    if (xdtype == 1)
-      v = __uint_as_float((uint32_t)static_cast<const uint16_t*>(x)[base + j] << 16);
-    else
-      v = static_cast<const float*>(x)[base + j];
-    xf[base + j] = v;
-    s += v;
-  }
-  s = warp_sum(s);
-  if (lane == 0) xs[e] = s;
+// 4-byte asynchronous copy global -> shared (cp.async), and the wait for all of
+// this thread's copies.
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Shared-memory plan of one block.
+struct DgPlan {
+  int ks, gps;   // group-range splits, groups per split
+  int wstride;   // words per staged row (>= the range's words, odd)
+  int sstride;   // scales / zeros per staged row (>= gps, odd)
+  size_t smem;
+};
+
+static size_t dg_smem(int wstride, int sstride, int gps, int B) {
+  return (size_t)DG_ROWS * wstride * 4 + 2 * (size_t)DG_ROWS * sstride * 4 + (size_t)(gps + 1) * 4 +
+         (size_t)B * gps * 4 + (size_t)DG_WARPS * B * DG_ROWS * 4;
 }
 
-// A[bb] += sum_j x[bb][j] f_j over the group's G codes (BITS each) in buf.
-template <int G, int BITS>
-__device__ __forceinline__ void dg_group(const uint32_t (&buf)[G / 4], const float* __restrict__ xg, int64_t n, int B,
-                                         float (&A)[DG_MAXB]) {
+// A range of groups holds at most its groups' full-row share of words when the
+// allocation is the usual one (rw words per row in all); widths up to 8 bits
+// bound it in any case.
+static DgPlan dg_plan(int64_t n, int group, int avg_bits, int B) {
+  const int k = (int)(n / group);
+  const int64_t rw = n * avg_bits / 32;
+  DgPlan pl{};
+  for (int ks = 1;; ++ks) {
+    const int gps = (k + ks - 1) / ks;
+    const int64_t wmax = std::min<int64_t>((int64_t)gps * group / 4, rw);
+    pl.ks = ks;
+    pl.gps = gps;
+    pl.wstride = (int)(wmax | 1);
+    pl.sstride = gps | 1;
+    pl.smem = dg_smem(pl.wstride, pl.sstride, gps, B);
+    if (pl.smem <= DG_SMEM_MAX || gps == 1) break;
+  }
+  return pl;
+}
+
+// A[bb] += sum_j x[bb][j] f_j over 32 consecutive codes of BITS bits each, held
+// in w[0 .. BITS) (32 codes of b bits are exactly b words); x fp32 or bf16.
+template <int BITS, int MB>
+__device__ __forceinline__ void dg_unit(const uint32_t (&w)[8], const void* __restrict__ x, bool xbf, int64_t col,
+                                        int64_t n, int B, float (&A)[MB]) {
 #pragma unroll
-  for (int j4 = 0; j4 < G; j4 += 4) {
+  for (int j4 = 0; j4 < 32; j4 += 4) {
     float f[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -65,15 +88,23 @@ __device__ __forceinline__ void dg_group(const uint32_t (&buf)[G / 4], const flo
       const int pos = (j4 + u) * BITS, wi = pos >> 5, off = pos & 31;
       uint32_t v;
       if (off + BITS <= 32)
-        v = buf[wi] >> off;
+        v = w[wi] >> off;
       else
-        v = __funnelshift_r(buf[wi], buf[wi + 1], off);
+        v = __funnelshift_r(w[wi], w[wi + 1], off);
       f[u] = __uint_as_float(((v & kMask) << (23 - BITS)) | 0x3F800000u);
     }
 #pragma unroll
-    for (int bb = 0; bb < DG_MAXB; ++bb)
+    for (int bb = 0; bb < MB; ++bb)
       if (bb < B) {
-        const float4 xv = *reinterpret_cast<const float4*>(xg + (int64_t)bb * n + j4);
+        const int64_t e = (int64_t)bb * n + col + j4;
+        float4 xv;
+        if (xbf) {
+          const uint2 h = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(x) + e);
+          xv = make_float4(__uint_as_float(h.x << 16), __uint_as_float(h.x & 0xFFFF0000u),
+                           __uint_as_float(h.y << 16), __uint_as_float(h.y & 0xFFFF0000u));
+        } else {
+          xv = *reinterpret_cast<const float4*>(static_cast<const float*>(x) + e);
+        }
         A[bb] = fmaf(xv.x, f[0], A[bb]);
         A[bb] = fmaf(xv.y, f[1], A[bb]);
         A[bb] = fmaf(xv.z, f[2], A[bb]);
@@ -82,63 +113,151 @@ __device__ __forceinline__ void dg_group(const uint32_t (&buf)[G / 4], const flo
   }
 }
 
-template <int G>
+template <int G, int MB>
 __global__ void __launch_bounds__(DG_WARPS * 32)
 dg_kernel(const uint32_t* __restrict__ codes, int64_t m, int64_t rw, const uint8_t* __restrict__ bits,
-          const float* __restrict__ scale, const float* __restrict__ zero, int k,
-          const float* __restrict__ xf, const float* __restrict__ xs, int B, int64_t n, int gps,
-          float* __restrict__ part) {
-  constexpr int NW = G / 4;  // words of a group at 8 bits, the widest
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t rb = (int64_t)blockIdx.x * DG_WARPS + warp;
-  const int64_t row = rb * 32 + lane;
-  const bool valid = row < m;
-  const int c0 = blockIdx.y * gps, c1 = (c0 + gps < k) ? c0 + gps : k;
-  float acc[DG_MAXB];
+          const float* __restrict__ scale, const float* __restrict__ zero, int k, const void* __restrict__ x,
+          int xdtype, int B, int64_t n, int gps, int wstride, int sstride, float* __restrict__ out) {
+  constexpr int SU = G / 32;  // 32-code sub-units per group
+  extern __shared__ uint32_t dsm[];
+  uint32_t* wsm = dsm;                                             // [32 rows][wstride] words
+  float* ssm = reinterpret_cast<float*>(wsm + DG_ROWS * wstride);  // [32][sstride] scales
+  float* zsm = ssm + DG_ROWS * sstride;                            // [32][sstride] zeros
+  int* woff = reinterpret_cast<int*>(zsm + DG_ROWS * sstride);     // [gps + 1] word offsets in the range
+  float* xsm = reinterpret_cast<float*>(woff + gps + 1);           // [B][gps] group sums of x
+  float* red = xsm + B * gps;                                      // [warps][B][32]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t r0 = (int64_t)blockIdx.x * DG_ROWS;
+  const int c0 = blockIdx.y * gps, c1 = (c0 + gps < k) ? c0 + gps : k, nc = c1 - c0;
+  const bool xbf = xdtype == 1;
+  // word offsets: the range's start (SU times the earlier groups' bits) and a
+  // prefix sum over the range
+  if (warp == 0) {
+    int before = 0;
+    for (int c = lane; c < c0; c += 32) before += bits[c];
 #pragma unroll
-  for (int bb = 0; bb < DG_MAXB; ++bb) acc[bb] = 0.f;
-  const uint32_t* rowp = codes + (valid ? row : 0) * rw;
-  // word offset of group c0 in a row: (G / 32) * sum of the earlier groups' bits,
-  // summed by the warp's lanes (the same on every lane); later groups add theirs
-  int before = 0;
-  for (int c = lane; c < c0; c += 32) before += bits[c];
+    for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+    int run = SU * before;
+    for (int cb = 0; cb < nc; cb += 32) {
+      const int c = cb + lane;
+      const int v = c < nc ? SU * (int)bits[c0 + c] : 0;
+      int incl = v;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
-  int ws = (G / 32) * before;
-  for (int c = c0; c < c1; ws += (G / 32) * bits[c], ++c) {
-    const int b = bits[c];
-    const int nw = (G / 32) * b;
-    uint32_t buf[NW];
-#pragma unroll
-    for (int u = 0; u < NW; ++u) buf[u] = (valid && u < nw && ws + u < rw) ? rowp[ws + u] : 0u;
-    float A[DG_MAXB];
-#pragma unroll
-    for (int bb = 0; bb < DG_MAXB; ++bb) A[bb] = 0.f;
-    const float* xg = xf + (int64_t)c * G;
-    switch (b) {
-      case 1: dg_group<G, 1>(buf, xg, n, B, A); break;
-      case 2: dg_group<G, 2>(buf, xg, n, B, A); break;
-      case 3: dg_group<G, 3>(buf, xg, n, B, A); break;
-      case 4: dg_group<G, 4>(buf, xg, n, B, A); break;
-      case 5: dg_group<G, 5>(buf, xg, n, B, A); break;
-      case 6: dg_group<G, 6>(buf, xg, n, B, A); break;
-      case 7: dg_group<G, 7>(buf, xg, n, B, A); break;
-      case 8: dg_group<G, 8>(buf, xg, n, B, A); break;
-      default: continue;  // not a valid width (the caller's precondition): the group adds nothing
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      if (c < nc) woff[c] = run + incl - v;
+      run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    const float s = valid ? scale[row * k + c] : 0.f, z = valid ? zero[row * k + c] : 0.f;
+    if (lane == 0) woff[nc] = run;
+  }
+  // scales and zeros of the 32 rows, copied asynchronously (consecutive threads:
+  // consecutive groups of a row); rows past m read as zero
+  for (int e = tid; e < DG_ROWS * nc; e += DG_WARPS * 32) {
+    const int r = e / nc, c = e - r * nc;
+    if (r0 + r < m) {
+      cp_async4(ssm + r * sstride + c, scale + (r0 + r) * k + c0 + c);
+      cp_async4(zsm + r * sstride + c, zero + (r0 + r) * k + c0 + c);
+    } else {
+      ssm[r * sstride + c] = 0.f;
+      zsm[r * sstride + c] = 0.f;
+    }
+  }
+  // group sums of x over the range: a thread per (batch row, group), 16-byte loads
+  for (int e = tid; e < B * nc; e += DG_WARPS * 32) {
+    const int bb = e / nc, c = e - bb * nc;
+    const int64_t base = (int64_t)bb * n + (int64_t)(c0 + c) * G;
+    float s0 = 0.f, s1 = 0.f;
+    if (xbf) {
+      const uint4* xp = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + base);
+#pragma unroll
+      for (int j = 0; j < G / 8; ++j) {
+        const uint4 v = xp[j];
+        s0 += __uint_as_float(v.x << 16) + __uint_as_float(v.x & 0xFFFF0000u) + __uint_as_float(v.y << 16) +
+              __uint_as_float(v.y & 0xFFFF0000u);
+        s1 += __uint_as_float(v.z << 16) + __uint_as_float(v.z & 0xFFFF0000u) + __uint_as_float(v.w << 16) +
+              __uint_as_float(v.w & 0xFFFF0000u);
+      }
+    } else {
+      const float4* xp = reinterpret_cast<const float4*>(static_cast<const float*>(x) + base);
+#pragma unroll
+      for (int j = 0; j < G / 4; j += 2) {
+        const float4 v = xp[j], w2 = xp[j + 1];
+        s0 += (v.x + v.y) + (v.z + v.w);
+        s1 += (w2.x + w2.y) + (w2.z + w2.w);
+      }
+    }
+    xsm[bb * gps + c] = s0 + s1;
+  }
+  __syncthreads();
+  // the rows' words of the range, copied asynchronously (consecutive threads:
+  // consecutive words of a row); words past the staged stride (an allocation
+  // that does not fill its rows the usual way) are not read
+  const int w0 = woff[0];
+  const int nw = min(woff[nc] - w0, wstride);
+  for (int e = tid; e < DG_ROWS * nw; e += DG_WARPS * 32) {
+    const int r = e / nw, w = e - r * nw;
+    const int64_t wi = (int64_t)w0 + w;
+    if (r0 + r < m && wi < rw)
+      cp_async4(wsm + r * wstride + w, codes + (r0 + r) * rw + wi);
+    else
+      wsm[r * wstride + w] = 0u;
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  // decode: warp w takes groups w, w + 8, ... of the range; lane = row
+  float acc[MB];
+#pragma unroll
+  for (int bb = 0; bb < MB; ++bb) acc[bb] = 0.f;
+  const uint32_t* myw = wsm + lane * wstride;
+  for (int c = warp; c < nc; c += DG_WARPS) {
+    const int b = bits[c0 + c];
+    const int wl = woff[c] - w0;  // the group's first word in the staged row
+    if (b < 1 || b > 8 || wl + SU * b > nw) continue;  // not a valid width or beyond the staged words: adds nothing
+    float A[MB];
+#pragma unroll
+    for (int bb = 0; bb < MB; ++bb) A[bb] = 0.f;
+    const int64_t col = (int64_t)(c0 + c) * G;
+#pragma unroll
+    for (int j = 0; j < SU; ++j) {
+      uint32_t w[8];
+      const int wo = wl + j * b;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) w[u] = u < b ? myw[wo + u] : 0u;
+      switch (b) {
+        case 1: dg_unit<1, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
+        case 2: dg_unit<2, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
+        case 3: dg_unit<3, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
+        case 4: dg_unit<4, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
+        case 5: dg_unit<5, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
+        case 6: dg_unit<6, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
+        case 7: dg_unit<7, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
+        default: dg_unit<8, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
+      }
+    }
+    const float s = ssm[lane * sstride + c], z = zsm[lane * sstride + c];
     const float p2 = (float)(1 << b);
 #pragma unroll
-    for (int bb = 0; bb < DG_MAXB; ++bb)
+    for (int bb = 0; bb < MB; ++bb)
       if (bb < B) {
-        const float xsum = xs[bb * k + c];
+        const float xsum = xsm[bb * gps + c];
         acc[bb] = fmaf(s, fmaf(p2, A[bb] - xsum, -z * xsum), acc[bb]);
       }
   }
-  if (valid)
 #pragma unroll
-    for (int bb = 0; bb < DG_MAXB; ++bb)
-      if (bb < B) part[((int64_t)blockIdx.y * B + bb) * m + row] = acc[bb];
+  for (int bb = 0; bb < MB; ++bb)
+    if (bb < B) red[(warp * B + bb) * 32 + lane] = acc[bb];
+  __syncthreads();
+  // the warps' sums in order; a single range writes y, several write partials [split][B][m]
+  for (int e = tid; e < B * DG_ROWS; e += DG_WARPS * 32) {
+    const int bb = e / DG_ROWS, r = e - bb * DG_ROWS;
+    if (r0 + r >= m) continue;
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < DG_WARPS; ++w) s += red[(w * B + bb) * 32 + r];
+    out[((int64_t)blockIdx.y * B + bb) * m + r0 + r] = s;
+  }
 }
 
 __global__ void dg_reduce_kernel(const float* __restrict__ part, int ks, int B, int64_t m, float* __restrict__ y) {
@@ -149,44 +268,52 @@ __global__ void dg_reduce_kernel(const float* __restrict__ part, int ks, int B, 
   y[e] = s;
 }
 
-// Splits of the groups per row block: enough warps for about 16 per SM.
-static int dg_splits(int64_t m, int k, int num_sms) {
-  const int64_t rbw = (m + 31) / 32;
-  int64_t ks = ((int64_t)num_sms * 16 + rbw - 1) / rbw;
-  if (ks > k) ks = k;
-  if (ks < 1) ks = 1;
-  return (int)ks;
-}
-
-size_t dg_workspace_bytes(int64_t m, int64_t n, int group, int64_t B, int num_sms) {
-  const int k = (int)(n / group);
-  const int ks = dg_splits(m, k, num_sms);
-  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
-  return al((size_t)B * n * 4) + al((size_t)B * k * 4) + al((size_t)ks * B * m * 4);
+size_t dg_workspace_bytes(int64_t m, int64_t n, int group, int avg_bits, int64_t B) {
+  const DgPlan pl = dg_plan(n, group, avg_bits, (int)B);
+  return pl.ks > 1 ? (size_t)pl.ks * B * m * 4 : 0;
 }
 
 cudaError_t launch_dequant_gemv(const uint32_t* codes, const uint8_t* bits, const float* scale, const float* zero,
                                 int64_t m, int64_t n, int group, int avg_bits, const void* x, int xdtype, int B,
-                                float* y, uint8_t* ws, int num_sms, cudaStream_t s) {
+                                float* y, uint8_t* ws, cudaStream_t s) {
   const int k = (int)(n / group);
   const int64_t rw = n * avg_bits / 32;
-  const int ks = dg_splits(m, k, num_sms);
-  const int gps = (k + ks - 1) / ks;
-  const int ksr = (k + gps - 1) / gps;  // splits actually holding groups
-  auto al = [](size_t v) { return (v + 255) & ~size_t(255); };
-  float* xf = reinterpret_cast<float*>(ws);
-  float* xs = reinterpret_cast<float*>(ws + al((size_t)B * n * 4));
-  float* part = reinterpret_cast<float*>(ws + al((size_t)B * n * 4) + al((size_t)B * k * 4));
-  dg_prep_kernel<<<(B * k + 7) / 8, 256, 0, s>>>(k, group, x, xdtype, B, n, xf, xs);
-  const dim3 grid((unsigned)(((m + 31) / 32 + DG_WARPS - 1) / DG_WARPS), (unsigned)ksr);
+  const DgPlan pl = dg_plan(n, group, avg_bits, B);
+  if (pl.smem > 227 * 1024) return cudaErrorInvalidValue;
+  float* out = pl.ks > 1 ? reinterpret_cast<float*>(ws) : y;
+  const int mb = B <= 1 ? 1 : (B <= 2 ? 2 : (B <= 4 ? 4 : 8));
+  const dim3 grid((unsigned)((m + DG_ROWS - 1) / DG_ROWS), (unsigned)pl.ks);
+  cudaError_t e = cudaSuccess;
+#define SLIM_DG(G, MB)                                                                                           \
+  do {                                                                                                           \
+    if (pl.smem > 48 * 1024)                                                                                     \
+      e = cudaFuncSetAttribute(dg_kernel<G, MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);     \
+    if (e == cudaSuccess)                                                                                        \
+      dg_kernel<G, MB><<<grid, DG_WARPS * 32, pl.smem, s>>>(codes, m, rw, bits, scale, zero, k, x, xdtype, B, n, \
+                                                            pl.gps, pl.wstride, pl.sstride, out);                \
+  } while (0)
+#define SLIM_DG_B(G)               \
+  switch (mb) {                    \
+    case 1: SLIM_DG(G, 1); break;  \
+    case 2: SLIM_DG(G, 2); break;  \
+    case 4: SLIM_DG(G, 4); break;  \
+    default: SLIM_DG(G, 8); break; \
+  }
   switch (group) {
-    case 32: dg_kernel<32><<<grid, DG_WARPS * 32, 0, s>>>(codes, m, rw, bits, scale, zero, k, xf, xs, B, n, gps, part); break;
-    case 64: dg_kernel<64><<<grid, DG_WARPS * 32, 0, s>>>(codes, m, rw, bits, scale, zero, k, xf, xs, B, n, gps, part); break;
-    case 128: dg_kernel<128><<<grid, DG_WARPS * 32, 0, s>>>(codes, m, rw, bits, scale, zero, k, xf, xs, B, n, gps, part); break;
+    case 32: SLIM_DG_B(32); break;
+    case 64: SLIM_DG_B(64); break;
+    case 128: SLIM_DG_B(128); break;
     default: return cudaErrorInvalidValue;
   }
-  dg_reduce_kernel<<<(unsigned)((B * m + 255) / 256), 256, 0, s>>>(part, ksr, B, m, y);
-  count_launches(3);
+#undef SLIM_DG_B
+#undef SLIM_DG
+  if (e != cudaSuccess) return e;
+  int launches = 1;
+  if (pl.ks > 1) {
+    dg_reduce_kernel<<<(unsigned)((B * m + 255) / 256), 256, 0, s>>>(out, pl.ks, B, m, y);
+    ++launches;
+  }
+  count_launches(launches);
   return cudaGetLastError();
 }
 

@@ -348,6 +348,11 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -605,15 +610,15 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
             sqp = f2_fma(dd, dd, sqp);
           }
         } else {
+          float dm = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+#pragma unroll
+          for (int j = 3; j < 63; j += 2) dm = fmax3(dm, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+          dm = fmaxf(dm, __uint_as_float(v[63]));
           // A quantized output far above its full-precision value (d above about
           // 44 in output units) would overflow e^d in fp32. The thread's largest
           // exponent decides a shift csh, a multiple of 32 that keeps every term
           // at most 2^64; it is 0 for ordinary layers, where e^(d log2(e) - 0)
           // is exactly the unshifted term.
-          float dm = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
-#pragma unroll
-          for (int j = 3; j < 63; j += 2) dm = fmax3(dm, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-          dm = fmaxf(dm, __uint_as_float(v[63]));
           const float c = dm * kC1 - 64.f;
           csh = c > 0.f ? 32.f * ceilf(c * (1.f / 32.f)) : 0.f;
           const uint64_t kc2 = f2_pack(kC1, kC1), nc = f2_pack(-csh, -csh);
@@ -761,8 +766,14 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           tmem_ld16(td + 16 * q, u);
           tc_wait_ld16(u);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            v[16 * q + j] = __float_as_uint(__fadd_rn(__uint_as_float(v[16 * q + j]), __uint_as_float(u[j])));
+          for (int j = 0; j < 16; j += 2) {
+            float x0, x1;
+            f2_unpack(f2_add(f2_pack(__uint_as_float(v[16 * q + j]), __uint_as_float(v[16 * q + j + 1])),
+                             f2_pack(__uint_as_float(u[j]), __uint_as_float(u[j + 1]))),
+                      x0, x1);
+            v[16 * q + j] = __float_as_uint(x0);
+            v[16 * q + j + 1] = __float_as_uint(x1);
+          }
         }
         release_early(step);
         if (!finish_step(step, 0.f)) { ok = false; break; }

@@ -77,7 +77,7 @@ _SIGS = {
     "slim_sqc": (i32, [vp, i64, i64, vp, vp, i32, i32, dbl, i32, vp, vp, vp, vp, vp]),
     "slim_gptq_workspace_bytes": (sz, [i64, i64]),
     "slim_gptq": (i32, [vp, i64, i64, vp, vp, i32, i32, dbl, i32, vp, vp, vp, vp, vp, sz, vp]),
-    "slim_dequant_gemv_workspace_bytes": (sz, [i64, i64, i32, i64]),
+    "slim_dequant_gemv_workspace_bytes": (sz, [i64, i64, i32, i32, i64]),
     "slim_dequant_gemv": (i32, [vp, vp, vp, vp, i64, i64, i32, i32, vp, i32, i64, vp, vp, sz, vp]),
     "slim_workspace_bytes": (sz, [i64, i64, i64, i32, i32, i32]),
     "slim_quantize_layer": (i32, [vp, i64, i64, vp, i32, i64, i32, i32, dbl, i32, vp, vp, vp, vp, vp, sz, vp]),

@@ -69,7 +69,7 @@ def test_dequant_gemv_is_asynchronous_and_repeatable():
     words, bits, scale, zero = quantized_layer(512, 1024, 128, 2, seed=9)
     dev = [torch.from_numpy(a).cuda() for a in (words.view(np.int32), bits, scale, zero)]
     x = torch.randn((2, 1024), device="cuda")
-    ws = torch.empty(slim._lib().slim_dequant_gemv_workspace_bytes(512, 1024, 128, 2), dtype=torch.uint8,
+    ws = torch.empty(max(256, slim._lib().slim_dequant_gemv_workspace_bytes(512, 1024, 128, 2, 2)), dtype=torch.uint8,
                      device="cuda")
     ys = [slim.slim_dequant_gemv(*dev, 128, 2, x, ws=ws) for _ in range(5)]
     torch.cuda.synchronize()
