@@ -32,7 +32,7 @@ namespace slim {
 
 constexpr int DG_WARPS = 8;
 constexpr int DG_ROWS = 32;
-constexpr size_t DG_SMEM_MAX = 100 * 1024;  // two blocks per SM
+constexpr size_t DG_SMEM_MAX = 110 * 1024;  // two blocks per SM
 
 // 4-byte asynchronous copy global -> shared (cp.async), and the wait for all of
 // this thread's copies.
@@ -49,9 +49,9 @@ struct DgPlan {
   size_t smem;
 };
 
-static size_t dg_smem(int wstride, int sstride, int gps, int B) {
+static size_t dg_smem(int wstride, int sstride, int gps, int group, int B) {
   return (size_t)DG_ROWS * wstride * 4 + 2 * (size_t)DG_ROWS * sstride * 4 + (size_t)(gps + 1) * 4 +
-         (size_t)B * gps * 4 + (size_t)DG_WARPS * B * DG_ROWS * 4;
+         (size_t)B * gps * 4 + (size_t)DG_WARPS * B * DG_ROWS * 4 + (size_t)B * gps * group * 4;
 }
 
 // A range of groups holds at most its groups' full-row share of words when the
@@ -68,43 +68,42 @@ static DgPlan dg_plan(int64_t n, int group, int avg_bits, int B) {
     pl.gps = gps;
     pl.wstride = (int)(wmax | 1);
     pl.sstride = gps | 1;
-    pl.smem = dg_smem(pl.wstride, pl.sstride, gps, B);
+    pl.smem = dg_smem(pl.wstride, pl.sstride, gps, group, B);
     if (pl.smem <= DG_SMEM_MAX || gps == 1) break;
   }
   return pl;
 }
 
-// A[bb] += sum_j x[bb][j] f_j over 32 consecutive codes of BITS bits each, held
-// in w[0 .. BITS) (32 codes of b bits are exactly b words); x fp32 or bf16.
+// A[bb] += sum_j x[bb][j] f_j over 32 consecutive codes of BITS bits each: the
+// BITS words at wp (32 codes of b bits are exactly b words), x (fp32) at xr +
+// bb * xstride. Code j sits at bit j*BITS; one shift brings it to bit 23 - BITS
+// and one three-input logic op keeps it and sets the exponent of 1.0f.
 template <int BITS, int MB>
-__device__ __forceinline__ void dg_unit(const uint32_t (&w)[8], const void* __restrict__ x, bool xbf, int64_t col,
-                                        int64_t n, int B, float (&A)[MB]) {
+__device__ __forceinline__ void dg_unit(const uint32_t* __restrict__ wp, const float* __restrict__ xr, int xstride,
+                                        int B, float (&A)[MB]) {
+  uint32_t w[BITS];
+#pragma unroll
+  for (int u = 0; u < BITS; ++u) w[u] = wp[u];
+  constexpr uint32_t kField = ((1u << BITS) - 1) << (23 - BITS);
 #pragma unroll
   for (int j4 = 0; j4 < 32; j4 += 4) {
     float f[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      constexpr int kMask = (1 << BITS) - 1;
       const int pos = (j4 + u) * BITS, wi = pos >> 5, off = pos & 31;
       uint32_t v;
-      if (off + BITS <= 32)
-        v = w[wi] >> off;
-      else
-        v = __funnelshift_r(w[wi], w[wi + 1], off);
-      f[u] = __uint_as_float(((v & kMask) << (23 - BITS)) | 0x3F800000u);
+      if (off + BITS <= 32) {
+        constexpr int kTo = 23 - BITS;  // the field moves from bit off to bit kTo
+        v = off <= kTo ? w[wi] << (kTo - off) : w[wi] >> (off - kTo);
+      } else {
+        v = __funnelshift_r(w[wi], w[wi + 1], off) << (23 - BITS);
+      }
+      f[u] = __uint_as_float((v & kField) | 0x3F800000u);
     }
 #pragma unroll
     for (int bb = 0; bb < MB; ++bb)
       if (bb < B) {
-        const int64_t e = (int64_t)bb * n + col + j4;
-        float4 xv;
-        if (xbf) {
-          const uint2 h = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(x) + e);
-          xv = make_float4(__uint_as_float(h.x << 16), __uint_as_float(h.x & 0xFFFF0000u),
-                           __uint_as_float(h.y << 16), __uint_as_float(h.y & 0xFFFF0000u));
-        } else {
-          xv = *reinterpret_cast<const float4*>(static_cast<const float*>(x) + e);
-        }
+        const float4 xv = *reinterpret_cast<const float4*>(xr + bb * xstride + j4);
         A[bb] = fmaf(xv.x, f[0], A[bb]);
         A[bb] = fmaf(xv.y, f[1], A[bb]);
         A[bb] = fmaf(xv.z, f[2], A[bb]);
@@ -120,12 +119,15 @@ dg_kernel(const uint32_t* __restrict__ codes, int64_t m, int64_t rw, const uint8
           int xdtype, int B, int64_t n, int gps, int wstride, int sstride, float* __restrict__ out) {
   constexpr int SU = G / 32;  // 32-code sub-units per group
   extern __shared__ uint32_t dsm[];
+  // (the regions whose sizes are multiples of 4 words come first, so that the
+  // 16-byte accesses to x stay aligned)
   uint32_t* wsm = dsm;                                             // [32 rows][wstride] words
   float* ssm = reinterpret_cast<float*>(wsm + DG_ROWS * wstride);  // [32][sstride] scales
   float* zsm = ssm + DG_ROWS * sstride;                            // [32][sstride] zeros
-  int* woff = reinterpret_cast<int*>(zsm + DG_ROWS * sstride);     // [gps + 1] word offsets in the range
-  float* xsm = reinterpret_cast<float*>(woff + gps + 1);           // [B][gps] group sums of x
-  float* red = xsm + B * gps;                                      // [warps][B][32]
+  float* xfs = zsm + DG_ROWS * sstride;                            // [B][gps * G] x of the range, fp32
+  float* red = xfs + B * gps * G;                                  // [warps][B][32]
+  float* xsm = red + DG_WARPS * B * DG_ROWS;                       // [B][gps] group sums of x
+  int* woff = reinterpret_cast<int*>(xsm + B * gps);               // [gps + 1] word offsets in the range
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t r0 = (int64_t)blockIdx.x * DG_ROWS;
   const int c0 = blockIdx.y * gps, c1 = (c0 + gps < k) ? c0 + gps : k, nc = c1 - c0;
@@ -154,39 +156,45 @@ dg_kernel(const uint32_t* __restrict__ codes, int64_t m, int64_t rw, const uint8
   }
   // scales and zeros of the 32 rows, copied asynchronously (consecutive threads:
   // consecutive groups of a row); rows past m read as zero
-  for (int e = tid; e < DG_ROWS * nc; e += DG_WARPS * 32) {
-    const int r = e / nc, c = e - r * nc;
-    if (r0 + r < m) {
-      cp_async4(ssm + r * sstride + c, scale + (r0 + r) * k + c0 + c);
-      cp_async4(zsm + r * sstride + c, zero + (r0 + r) * k + c0 + c);
+  for (int r = warp; r < DG_ROWS; r += DG_WARPS)
+    for (int c = lane; c < nc; c += 32) {
+      if (r0 + r < m) {
+        cp_async4(ssm + r * sstride + c, scale + (r0 + r) * k + c0 + c);
+        cp_async4(zsm + r * sstride + c, zero + (r0 + r) * k + c0 + c);
+      } else {
+        ssm[r * sstride + c] = 0.f;
+        zsm[r * sstride + c] = 0.f;
+      }
+    }
+  // x of the range as fp32 (bf16 widened exactly), 16-byte loads
+  const int xstride = gps * G, ncol = nc * G;
+  for (int e = tid; e < B * (ncol / 8); e += DG_WARPS * 32) {
+    const int bb = e / (ncol / 8), j = (e - bb * (ncol / 8)) * 8;
+    const int64_t src = (int64_t)bb * n + (int64_t)c0 * G + j;
+    float* d = xfs + bb * xstride + j;
+    if (xbf) {
+      const uint4 v = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + src);
+      *reinterpret_cast<float4*>(d) = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
+                                                  __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
+      *reinterpret_cast<float4*>(d + 4) = make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xFFFF0000u),
+                                                      __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xFFFF0000u));
     } else {
-      ssm[r * sstride + c] = 0.f;
-      zsm[r * sstride + c] = 0.f;
+      const float4* xp = reinterpret_cast<const float4*>(static_cast<const float*>(x) + src);
+      *reinterpret_cast<float4*>(d) = xp[0];
+      *reinterpret_cast<float4*>(d + 4) = xp[1];
     }
   }
-  // group sums of x over the range: a thread per (batch row, group), 16-byte loads
+  __syncthreads();
+  // group sums of x over the range: a thread per (batch row, group)
   for (int e = tid; e < B * nc; e += DG_WARPS * 32) {
     const int bb = e / nc, c = e - bb * nc;
-    const int64_t base = (int64_t)bb * n + (int64_t)(c0 + c) * G;
+    const float4* xp = reinterpret_cast<const float4*>(xfs + bb * xstride + c * G);
     float s0 = 0.f, s1 = 0.f;
-    if (xbf) {
-      const uint4* xp = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + base);
 #pragma unroll
-      for (int j = 0; j < G / 8; ++j) {
-        const uint4 v = xp[j];
-        s0 += __uint_as_float(v.x << 16) + __uint_as_float(v.x & 0xFFFF0000u) + __uint_as_float(v.y << 16) +
-              __uint_as_float(v.y & 0xFFFF0000u);
-        s1 += __uint_as_float(v.z << 16) + __uint_as_float(v.z & 0xFFFF0000u) + __uint_as_float(v.w << 16) +
-              __uint_as_float(v.w & 0xFFFF0000u);
-      }
-    } else {
-      const float4* xp = reinterpret_cast<const float4*>(static_cast<const float*>(x) + base);
-#pragma unroll
-      for (int j = 0; j < G / 4; j += 2) {
-        const float4 v = xp[j], w2 = xp[j + 1];
-        s0 += (v.x + v.y) + (v.z + v.w);
-        s1 += (w2.x + w2.y) + (w2.z + w2.w);
-      }
+    for (int j = 0; j < G / 4; j += 2) {
+      const float4 v = xp[j], w2 = xp[j + 1];
+      s0 += (v.x + v.y) + (v.z + v.w);
+      s1 += (w2.x + w2.y) + (w2.z + w2.w);
     }
     xsm[bb * gps + c] = s0 + s1;
   }
@@ -196,13 +204,15 @@ dg_kernel(const uint32_t* __restrict__ codes, int64_t m, int64_t rw, const uint8
   // that does not fill its rows the usual way) are not read
   const int w0 = woff[0];
   const int nw = min(woff[nc] - w0, wstride);
-  for (int e = tid; e < DG_ROWS * nw; e += DG_WARPS * 32) {
-    const int r = e / nw, w = e - r * nw;
-    const int64_t wi = (int64_t)w0 + w;
-    if (r0 + r < m && wi < rw)
-      cp_async4(wsm + r * wstride + w, codes + (r0 + r) * rw + wi);
-    else
-      wsm[r * wstride + w] = 0u;
+  for (int r = warp; r < DG_ROWS; r += DG_WARPS) {
+    const bool row_ok = r0 + r < m;
+    const uint32_t* src = codes + (row_ok ? r0 + r : 0) * rw + w0;
+    for (int w = lane; w < nw; w += 32) {
+      if (row_ok && (int64_t)w0 + w < rw)
+        cp_async4(wsm + r * wstride + w, src + w);
+      else
+        wsm[r * wstride + w] = 0u;
+    }
   }
   cp_async_wait_all();
   __syncthreads();
@@ -218,26 +228,23 @@ dg_kernel(const uint32_t* __restrict__ codes, int64_t m, int64_t rw, const uint8
     float A[MB];
 #pragma unroll
     for (int bb = 0; bb < MB; ++bb) A[bb] = 0.f;
-    const int64_t col = (int64_t)(c0 + c) * G;
+    const float* xr = xfs + c * G;
 #pragma unroll
     for (int j = 0; j < SU; ++j) {
-      uint32_t w[8];
-      const int wo = wl + j * b;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) w[u] = u < b ? myw[wo + u] : 0u;
+      const uint32_t* wp = myw + wl + j * b;
       switch (b) {
-        case 1: dg_unit<1, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
-        case 2: dg_unit<2, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
-        case 3: dg_unit<3, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
-        case 4: dg_unit<4, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
-        case 5: dg_unit<5, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
-        case 6: dg_unit<6, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
-        case 7: dg_unit<7, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
-        default: dg_unit<8, MB>(w, x, xbf, col + 32 * j, n, B, A); break;
+        case 1: dg_unit<1, MB>(wp, xr + 32 * j, xstride, B, A); break;
+        case 2: dg_unit<2, MB>(wp, xr + 32 * j, xstride, B, A); break;
+        case 3: dg_unit<3, MB>(wp, xr + 32 * j, xstride, B, A); break;
+        case 4: dg_unit<4, MB>(wp, xr + 32 * j, xstride, B, A); break;
+        case 5: dg_unit<5, MB>(wp, xr + 32 * j, xstride, B, A); break;
+        case 6: dg_unit<6, MB>(wp, xr + 32 * j, xstride, B, A); break;
+        case 7: dg_unit<7, MB>(wp, xr + 32 * j, xstride, B, A); break;
+        default: dg_unit<8, MB>(wp, xr + 32 * j, xstride, B, A); break;
       }
     }
     const float s = ssm[lane * sstride + c], z = zsm[lane * sstride + c];
-    const float p2 = (float)(1 << b);
+    const float p2 = __int_as_float((127 + b) << 23);  // 2^b
 #pragma unroll
     for (int bb = 0; bb < MB; ++bb)
       if (bb < B) {

@@ -205,6 +205,7 @@ constexpr int SB_BN = 128;        // outputs per tile (one TMEM slot: y and d, 1
 constexpr int SB_BK = 64;         // K elements per box (128 bytes of fp16)
 constexpr int SB_BOX = SB_BM * SB_BK * 2;  // 16 KB
 constexpr int SB_STAGE = 4 * SB_BOX;       // X(token tile 0), X(token tile 1), B1, B2
+constexpr int kNarrowBox = SB_BM * 32 * 2;  // 128 rows x 32 fp16 columns: 8 KB (a group-32 step's boxes)
 constexpr int SB_BAND = 16;                // token-tile pairs per raster band
 constexpr int SB_MAX_K = 1024;
 constexpr int SB_EPI_WARPS = 16;           // warps 2..9 read slot 0, warps 10..17 slot 1 (two per row)
@@ -213,7 +214,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kC1 = kLog2e * kOpUnscale;  // exponent scale for accumulator (x 2^8) units
 
 struct SbaTmaps {
-  CUtensorMap x, wb, e0, dp, dm;
+  CUtensorMap x, wb, e0, dp, dm;  // 64-column boxes, 128-byte swizzle
+  CUtensorMap x32, dp32, dm32;     // 32-column boxes, 64-byte swizzle (candidate steps at group 32)
 };
 
 struct SbaParams {
@@ -427,6 +429,8 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
   const uint32_t tbase = *tslot;
   const int units = p.n_tp * p.n_ot;
   const int nA = *s_na;
+  // candidate steps at group 32 with bf16 X: one stage per step of 32-column boxes
+  const bool narrow = p.g == 32 && p.nsub == 2;
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
@@ -440,6 +444,26 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
         unit_decode(p, u, tp, ot);
         const int xrow0 = 2 * tp * SB_BM, xrow1 = xrow0 + SB_BM, brow = ot * SB_BN;
         for (int step = s_lo; step < s_hi && ok; ++step) {
+          if (narrow && step > 0) {
+            // the whole step in one stage: X of both groups for both token tiles,
+            // then the Dp / Dm boxes (hi, and lo for a split box), 8 KB each
+            const int cu = s_order[step - 1] * 32, cd = s_order[p.k - step] * 32;
+            const int su = s_split[cu >> 6], sd = s_split[cd >> 6];
+            if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, p.st, 200 + st)) { ok = false; break; }
+            uint8_t* sb = smem + st * SB_STAGE;
+            mbar_arrive_expect_tx(&full[st], (6 + su + sd) * kNarrowBox);
+            tma_load_2d(sb, &tm.x32, &full[st], cu, xrow0);
+            tma_load_2d(sb + kNarrowBox, &tm.x32, &full[st], cu, xrow1);
+            tma_load_2d(sb + 2 * kNarrowBox, &tm.x32, &full[st], cd, xrow0);
+            tma_load_2d(sb + 3 * kNarrowBox, &tm.x32, &full[st], cd, xrow1);
+            tma_load_2d(sb + 4 * kNarrowBox, &tm.dp32, &full[st], cu, brow);
+            tma_load_2d(sb + 5 * kNarrowBox, &tm.dm32, &full[st], cd, brow);
+            if (su) tma_load_2d(sb + 6 * kNarrowBox, &tm.dp32, &full[st], p.npad + cu, brow);
+            if (sd) tma_load_2d(sb + 7 * kNarrowBox, &tm.dm32, &full[st], p.npad + cd, brow);
+            ++it;
+            if (++st == S) { st = 0; ph ^= 1; }
+            continue;
+          }
           const ItemGeom geo = item_geom(p, s_order, s_split, nA, step);
           const int nch = geo.nch;
           for (int c = 0; c < nch; ++c) {
@@ -492,6 +516,44 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           if (!mbar_wait(&afree[0], (cnt & 1) ^ fpar, abort_flag, p.st, 220) ||
               !mbar_wait(&afree[1], (cnt & 1) ^ fpar, abort_flag, p.st, 221)) { ok = false; break; }
           tc_fence_after();
+          if (narrow && step > 0) {
+            // one stage: both groups' 32-column boxes (64-byte swizzle), the
+            // promoted group first, each as hi then lo, from a zero accumulator
+            const int su = s_split[(s_order[step - 1] * 32) >> 6], sd = s_split[(s_order[p.k - step] * 32) >> 6];
+            if (!mbar_wait(&full[st], ph, abort_flag, p.st, 230 + st)) { ok = false; break; }
+            tc_fence_after();
+            // box i of the stage at start address + i * 8 KB (= 512 in 16-byte units)
+            const uint64_t d0 = sdesc_sw64(smem_u32(smem) + (uint32_t)st * SB_STAGE);
+            constexpr uint64_t kNb16 = kNarrowBox / 16;
+#pragma unroll
+            for (int k16 = 0; k16 < 2; ++k16) {
+              tc_mma_f16(ty0 + 128, d0 + 2 * k16, d0 + 4 * kNb16 + 2 * k16, idesc, k16 > 0 ? 1u : 0u);
+              tc_mma_f16(ty1 + 128, d0 + kNb16 + 2 * k16, d0 + 4 * kNb16 + 2 * k16, idesc, k16 > 0 ? 1u : 0u);
+            }
+            if (su)
+#pragma unroll
+              for (int k16 = 0; k16 < 2; ++k16) {
+                tc_mma_f16(ty0 + 128, d0 + 2 * k16, d0 + 6 * kNb16 + 2 * k16, idesc, 1u);
+                tc_mma_f16(ty1 + 128, d0 + kNb16 + 2 * k16, d0 + 6 * kNb16 + 2 * k16, idesc, 1u);
+              }
+#pragma unroll
+            for (int k16 = 0; k16 < 2; ++k16) {
+              tc_mma_f16(ty0 + 128, d0 + 2 * kNb16 + 2 * k16, d0 + 5 * kNb16 + 2 * k16, idesc, 1u);
+              tc_mma_f16(ty1 + 128, d0 + 3 * kNb16 + 2 * k16, d0 + 5 * kNb16 + 2 * k16, idesc, 1u);
+            }
+            if (sd)
+#pragma unroll
+              for (int k16 = 0; k16 < 2; ++k16) {
+                tc_mma_f16(ty0 + 128, d0 + 2 * kNb16 + 2 * k16, d0 + 7 * kNb16 + 2 * k16, idesc, 1u);
+                tc_mma_f16(ty1 + 128, d0 + 3 * kNb16 + 2 * k16, d0 + 7 * kNb16 + 2 * k16, idesc, 1u);
+              }
+            tc_commit(&empty[st]);
+            if (++st == S) { st = 0; ph ^= 1; dcur = d_first; } else { dcur += kStage16; }
+            tc_commit(&afull[0]);
+            tc_commit(&afull[1]);
+            ++cnt;
+            continue;
+          }
           const ItemGeom geo = item_geom(p, s_order, s_split, nA, step);
           const int nch = geo.nch;
           // A shared-memory access by this thread while its MMAs are in flight
@@ -1154,6 +1216,9 @@ static cudaError_t launch_score(const SbaPlan& pl, int64_t m, int64_t n, int64_t
   ok = ok && make_tmap_f16(&tm.e0, pw + pl.off_e0, wcols, (uint64_t)m, SB_BK, SB_BN);
   ok = ok && make_tmap_f16(&tm.dp, pw + pl.off_dp, wcols, (uint64_t)m, SB_BK, SB_BN);
   ok = ok && make_tmap_f16(&tm.dm, pw + pl.off_dm, wcols, (uint64_t)m, SB_BK, SB_BN);
+  ok = ok && make_tmap_f16_sw64(&tm.x32, pw + pl.off_xc, (uint64_t)(n * pl.ksplit), (uint64_t)N, 32, SB_BM);
+  ok = ok && make_tmap_f16_sw64(&tm.dp32, pw + pl.off_dp, wcols, (uint64_t)m, 32, SB_BN);
+  ok = ok && make_tmap_f16_sw64(&tm.dm32, pw + pl.off_dm, wcols, (uint64_t)m, 32, SB_BN);
   if (!ok) return cudaErrorInvalidValue;
   SbaParams p;
   p.N = N; p.m = m; p.n = n; p.npad = pl.npad; p.g = group; p.k = pl.k; p.P = pl.P; p.ksplit = pl.ksplit;
