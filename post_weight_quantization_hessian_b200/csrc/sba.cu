@@ -688,7 +688,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
           // double-buffered (the load of the next one is in flight while this one
           // is consumed); the one-pass launch loads them one at a time. Same
           // arithmetic either way.
-          constexpr int NB = MODE == kSbaAll ? 1 : 2;
+          constexpr int NB = 2;
           uint32_t ev[NB][8];
           if (NB == 2) {
             tmem_ld8(ty, ev[0]);
@@ -857,7 +857,6 @@ __global__ void __launch_bounds__(SB_THREADS, 1) sba_score_kernel(const __grid_c
 __global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict__ part, int n_ot, int P, int64_t N,
                                                         int n_tt, int objective, int64_t m,
                                                         double* __restrict__ kl_part) {
-  extern __shared__ float s_f[];  // [n_ot][128] scale factors (one partial set per output tile)
   constexpr int QB = 8;  // candidates per pass
   __shared__ double red[4][QB];
   const int tt = blockIdx.x, r = threadIdx.x;
@@ -865,13 +864,14 @@ __global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict_
   const bool valid = (int64_t)tt * SB_BM + r < N;
   const float* base = part + (size_t)tt * n_ot * F * SB_BM + r;
   const bool mse = objective == 1;
+  // a tile's rescale factor to the token's overall maximum M, recomputed where
+  // it is used (the same value every time) rather than kept per tile
   float M = -3.0e38f;
   double Sy = 0.0;
   if (!mse) {
     for (int og = 0; og < n_ot; ++og) M = fmaxf(M, base[(size_t)og * F * SB_BM]);
     for (int og = 0; og < n_ot; ++og) {
       const float f = exp2f((base[(size_t)og * F * SB_BM] - M) * kLog2e);
-      s_f[og * SB_BM + r] = f;
       Sy += (double)base[(size_t)og * F * SB_BM + SB_BM] * (double)f;
     }
   }
@@ -885,8 +885,9 @@ __global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict_
     for (int j = 0; j < QB; ++j) sq[j] = a[j] = 0.0;
     bool shifted = false;
     for (int og = 0; og < n_ot; ++og) {
-      const double f = mse ? 1.0 : (double)s_f[og * SB_BM + r];
-      const float* bq = base + ((size_t)og * F + 2 + 2 * q0) * SB_BM;
+      const float* bt = base + (size_t)og * F * SB_BM;
+      const double f = mse ? 1.0 : (double)exp2f((bt[0] - M) * kLog2e);
+      const float* bq = bt + (size_t)(2 + 2 * q0) * SB_BM;
 #pragma unroll
       for (int j = 0; j < QB; ++j)
         if (j < nq) {
@@ -902,8 +903,9 @@ __global__ void __launch_bounds__(128) sba_merge_kernel(const float* __restrict_
 #pragma unroll
       for (int j = 0; j < QB; ++j) sq[j] = 0.0;
       for (int og = 0; og < n_ot; ++og) {
-        const double f = mse ? 1.0 : (double)s_f[og * SB_BM + r];
-        const float* bq = base + ((size_t)og * F + 2 + 2 * q0) * SB_BM;
+        const float* bt = base + (size_t)og * F * SB_BM;
+        const double f = mse ? 1.0 : (double)exp2f((bt[0] - M) * kLog2e);
+        const float* bq = bt + (size_t)(2 + 2 * q0) * SB_BM;
         for (int j = 0; j < QB; ++j)
           if (j < nq) {
             const float v = bq[(size_t)(2 * j) * SB_BM];
@@ -1261,12 +1263,7 @@ static cudaError_t launch_merge_final(const SbaPlan& pl, int64_t m, int64_t N, i
                                       cudaStream_t s) {
   float* part = reinterpret_cast<float*>(sw);
   double* klp = reinterpret_cast<double*>(sw + (pl.off_klp - pl.off_part));
-  const size_t msmem = (size_t)pl.n_ot * SB_BM * sizeof(float);
-  if (msmem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(sba_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
-    if (e != cudaSuccess) return e;
-  }
-  sba_merge_kernel<<<pl.n_tt, SB_BM, msmem, s>>>(part, pl.n_ot, pl.P, N, pl.n_tt, objective, m, klp);
+  sba_merge_kernel<<<pl.n_tt, SB_BM, 0, s>>>(part, pl.n_ot, pl.P, N, pl.n_tt, objective, m, klp);
   sba_final_kernel<<<1, 256, 0, s>>>(klp, pl.n_tt, pl.P, N, order, pl.k, avg_bits, kl, p_star, bits);
   count_launches(2);
   return cudaGetLastError();
