@@ -167,8 +167,8 @@ int slim_salience(const float* W, int64_t m, int64_t n, const double* h, int gro
  * point allocates nothing: its scratch is a fixed 256 KiB device array inside
  * the library (held on every GPU that loads the library until the process
  * exits), enough for n <= 32768 input columns; larger n returns SLIM_EINVAL.
- * The first call on a device looks up that array's device address, so make a
- * first call on each device before any stream capture. All calls on a device
+ * The first call on a device also looks up that array's device address. All
+ * calls on a device
  * share the array: calls that overlap on the GPU race and must be serialized
  * by the caller. The call waits for `stream` to drain before returning.
  */
