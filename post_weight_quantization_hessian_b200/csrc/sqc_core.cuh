@@ -35,8 +35,6 @@
 
 namespace slim {
 
-constexpr double kRintMagic = 6755399441055744.0;  // 1.5 * 2^52
-
 struct SqcChoice {
   double s, z0;  // scale tau* s0 and zero-point z0 (s = 1, z0 = -lo for a group of equal values)
   int t;         // chosen tau index
@@ -49,6 +47,7 @@ __device__ __forceinline__ SqcChoice sqc_choose(const double (&w)[G / 32], const
                                                 double lam, int n_tau, double* s_w, double* s_d, int lane) {
   constexpr int E = G / 32;
   const double qmax = (double)((1 << b) - 1);
+  const int qmaxi = (1 << b) - 1;
   double sum = 0.0, lo = 0.0, hi = 0.0;
 #pragma unroll
   for (int r = 0; r < E; ++r) {
@@ -116,11 +115,9 @@ __device__ __forceinline__ SqcChoice sqc_choose(const double (&w)[G / 32], const
         const double wj = s_w[j];
         const double q0 = __dmul_rn(wj, y);
         const double quot = fma(fma(-q0, s, wj), y, q0);   // = RN(wj / s)
-        // rint(v) (half to even) as (v + 1.5 2^52) - 1.5 2^52: exact for |v| < 2^51,
-        // which the quotients of weights by their group's scale stay far below;
-        // two fp64 adds instead of a conversion to integer and back
-        const double v = __dadd_rn(quot, z0);
-        const double q = fmin(fmax(__dsub_rn(__dadd_rn(v, kRintMagic), kRintMagic), 0.0), qmax);
+        int qi = __double2int_rn(__dadd_rn(quot, z0));     // round half to even, as rint
+        qi = qi < 0 ? 0 : (qi > qmaxi ? qmaxi : qi);
+        const double q = (double)qi;
         const double e = __dsub_rn(wj, __dmul_rn(s, __dsub_rn(q, z0)));
         return __dmul_rn(s_d[j], __dmul_rn(e, e));
       };
