@@ -280,6 +280,19 @@ size_t dg_workspace_bytes(int64_t m, int64_t n, int group, int avg_bits, int64_t
   return pl.ks > 1 ? (size_t)pl.ks * B * m * 4 : 0;
 }
 
+// The kernel instance's shared-memory limit raised to the plan's bound once per
+// device (a flag per instance and device), not on every call.
+template <int G, int MB>
+static cudaError_t dg_allow_smem() {
+  static std::atomic<uint64_t> done{0};
+  uint64_t bit = 0;
+  if (!attr_pending(done, bit)) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(dg_kernel<G, MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess) done.fetch_or(bit);
+  return e;
+}
+
 cudaError_t launch_dequant_gemv(const uint32_t* codes, const uint8_t* bits, const float* scale, const float* zero,
                                 int64_t m, int64_t n, int group, int avg_bits, const void* x, int xdtype, int B,
                                 float* y, uint8_t* ws, cudaStream_t s) {
@@ -293,8 +306,7 @@ cudaError_t launch_dequant_gemv(const uint32_t* codes, const uint8_t* bits, cons
   cudaError_t e = cudaSuccess;
 #define SLIM_DG(G, MB)                                                                                           \
   do {                                                                                                           \
-    if (pl.smem > 48 * 1024)                                                                                     \
-      e = cudaFuncSetAttribute(dg_kernel<G, MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);     \
+    if (pl.smem > 48 * 1024) e = dg_allow_smem<G, MB>();                                                         \
     if (e == cudaSuccess)                                                                                        \
       dg_kernel<G, MB><<<grid, DG_WARPS * 32, pl.smem, s>>>(codes, m, rw, bits, scale, zero, k, x, xdtype, B, n, \
                                                             pl.gps, pl.wstride, pl.sstride, out);                \
