@@ -103,30 +103,53 @@ __device__ __forceinline__ SqcChoice sqc_choose(const double (&w)[G / 32], const
   if (!deg) {
     best_e = __longlong_as_double(0x7ff0000000000000ll);  // +inf
     best_t = n_tau;
-    for (int t = lane; t < n_tau; t += 32) {
-      const double tau = (n_tau == 1) ? 1.0 : (1.0 - lam) + ((2.0 * lam) * (double)t) / (double)(n_tau - 1);
-      const double s = tau * s0;
-      const double y = 1.0 / s;
-      double es = 0.0, eu = 0.0;
+    // Two candidates per lane per pass (t0 = tb + lane, t1 = t0 + 32): their
+    // error sums are independent chains over the same elements, so the fp64
+    // add latency of one hides behind the other; each candidate's sum still
+    // runs in column order within the masked and the unmasked class. A lane
+    // without a second candidate (t1 >= n_tau) computes a discarded copy of
+    // its first.
+    const double step = (n_tau == 1) ? 0.0 : (2.0 * lam);
+    for (int tb = 0; tb < n_tau; tb += 64) {
+      const int t0 = tb + lane, t1 = t0 + 32;
+      if (t0 >= n_tau) break;  // (n_tau <= 256: whole passes of the warp stay uniform until here)
+      const bool two = t1 < n_tau;
+      const double tau0 = (n_tau == 1) ? 1.0 : (1.0 - lam) + (step * (double)t0) / (double)(n_tau - 1);
+      const double tau1 = two ? (1.0 - lam) + (step * (double)t1) / (double)(n_tau - 1) : tau0;
+      const double sa = tau0 * s0, sb = tau1 * s0;
+      const double ya = 1.0 / sa, yb = 1.0 / sb;
+      double esa = 0.0, eua = 0.0, esb = 0.0, eub = 0.0;
       // each rounding step of the definition separately (the _rn intrinsics
       // keep the compiler from contracting a product and a sum into an fma,
       // which would round once where the definition rounds twice)
-      auto term = [&](int j) {
-        const double wj = s_w[j];
+      auto term = [&](double wj, double dj, double s, double y) {
         const double q0 = __dmul_rn(wj, y);
         const double quot = fma(fma(-q0, s, wj), y, q0);   // = RN(wj / s)
         int qi = __double2int_rn(__dadd_rn(quot, z0));     // round half to even, as rint
         qi = qi < 0 ? 0 : (qi > qmaxi ? qmaxi : qi);
         const double q = (double)qi;
         const double e = __dsub_rn(wj, __dmul_rn(s, __dsub_rn(q, z0)));
-        return __dmul_rn(s_d[j], __dmul_rn(e, e));
+        return __dmul_rn(dj, __dmul_rn(e, e));
       };
-      for (int j = 0; j < ns; ++j) es = __dadd_rn(es, term(j));
-#pragma unroll 4
-      for (int j = ns; j < G; ++j) eu = __dadd_rn(eu, term(j));
-      double err = (nu > 0 ? eu / (double)nu : 0.0);
-      if (ns > 0) err = __dadd_rn(err, es / (double)ns);
-      if (err < best_e) { best_e = err; best_t = t; }
+      for (int j = 0; j < ns; ++j) {
+        const double wj = s_w[j], dj = s_d[j];
+        esa = __dadd_rn(esa, term(wj, dj, sa, ya));
+        esb = __dadd_rn(esb, term(wj, dj, sb, yb));
+      }
+#pragma unroll 2
+      for (int j = ns; j < G; ++j) {
+        const double wj = s_w[j], dj = s_d[j];
+        eua = __dadd_rn(eua, term(wj, dj, sa, ya));
+        eub = __dadd_rn(eub, term(wj, dj, sb, yb));
+      }
+      double erra = (nu > 0 ? eua / (double)nu : 0.0);
+      if (ns > 0) erra = __dadd_rn(erra, esa / (double)ns);
+      if (erra < best_e) { best_e = erra; best_t = t0; }
+      if (two) {
+        double errb = (nu > 0 ? eub / (double)nu : 0.0);
+        if (ns > 0) errb = __dadd_rn(errb, esb / (double)ns);
+        if (errb < best_e) { best_e = errb; best_t = t1; }
+      }
     }
     // warp argmin, ties to the smaller index
 #pragma unroll
