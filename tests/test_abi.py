@@ -93,3 +93,35 @@ def test_split_search_rejects_bad_chunks_before_any_launch(lib):
         rc = lib.slim_sba_search_split(0x1000, 256, 512, 0x2000, 1, 4096, 128, 2, 0x3000, None, None, 0x4000, chunk,
                                        None, 0, None)
         assert rc == 1, chunk
+
+
+def test_dequant_gemv_workspace_plan(lib):
+    """The GEMV's shared-memory plan on the host: one launch (no workspace) when a
+    block's 32 rows of words, scales, zeros and the batch's x fit; group ranges with
+    fixed-order partials (workspace ks * batch * m floats) when they do not."""
+    q = lib.slim_dequant_gemv_workspace_bytes
+    assert q(13824, 5120, 32, 2, 1) == 0        # the 13B up_proj at group 32, batch 1
+    assert q(4096, 4096, 128, 2, 1) == 0        # q_proj
+    # down_proj (b 3): 32 rows of 1032 words each do not fit beside the rest: group ranges
+    wd = q(4096, 11008, 128, 3, 1)
+    assert wd > 0 and wd % (4096 * 4) == 0 and wd // (4096 * 4) >= 2
+    w8 = q(13824, 5120, 32, 2, 8)               # batch 8: x of 8 rows no longer fits with the words
+    assert w8 > 0 and w8 % (8 * 13824 * 4) == 0 and w8 // (8 * 13824 * 4) >= 2
+    assert q(13824, 5120, 32, 2, 9) == 0        # batch above 8: not a valid call
+    assert q(13824, 5100, 32, 2, 1) == 0        # n not a multiple of the group
+
+
+def test_bench_traffic_record_follows_the_source():
+    """bench.py reports the committed DRAM bytes of the scoring kernel only while the
+    kernel's source is the one they were captured on."""
+    import os
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import bench
+    src = bench.source_hash("post_weight_quantization_hessian_b200/csrc/sba.cu",
+                            "post_weight_quantization_hessian_b200/csrc/common.cuh")
+    rec = bench.traffic_record("sba_score_kernel", "llama13b_up_proj_13824x5120_g32", src)
+    assert rec is not None and rec > 1e9
+    assert bench.traffic_record("sba_score_kernel", "llama13b_up_proj_13824x5120_g32", "0" * 16) is None
+    assert bench.traffic_record("sba_score_kernel", "no_such_workload", src) is None
