@@ -121,7 +121,13 @@ def test_bench_traffic_record_follows_the_source():
     import bench
     src = bench.source_hash("post_weight_quantization_hessian_b200/csrc/sba.cu",
                             "post_weight_quantization_hessian_b200/csrc/common.cuh")
+    import json
+    with open(os.path.join(root, "profiles", "traffic.json")) as f:
+        stored = json.load(f)["sba_score_kernel"]["llama13b_up_proj_13824x5120_g32"]
+    # the recorded bytes while the hash matches, nothing for any other source
+    assert bench.traffic_record("sba_score_kernel", "llama13b_up_proj_13824x5120_g32",
+                                stored["source_hash"]) == stored["bytes_per_launch"]
     rec = bench.traffic_record("sba_score_kernel", "llama13b_up_proj_13824x5120_g32", src)
-    assert rec is not None and rec > 1e9
+    assert rec == (stored["bytes_per_launch"] if src == stored["source_hash"] else None)
     assert bench.traffic_record("sba_score_kernel", "llama13b_up_proj_13824x5120_g32", "0" * 16) is None
     assert bench.traffic_record("sba_score_kernel", "no_such_workload", src) is None
