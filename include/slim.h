@@ -300,8 +300,11 @@ int slim_gptq(const float* W, int64_t m, int64_t n, const double* H, const uint8
  *   scale, zero  device m x k float32.
  *   x        device batch x n, row-major, float32 or bf16 (xdtype).
  *   y        device batch x m float32.
- * batch is 1..8. Arithmetic: fp32 (each code times x in one fma). The call is
- * asynchronous: it returns once the kernels are enqueued on `stream` (host-side
+ * batch is 1..8. Arithmetic: fp32. Per row, group c of width b and token,
+ * A = sum_j x_j (1 + q_j 2^-b) and xs = sum_j x_j, and y gains
+ * scale (2^b (A - xs) - zero xs), which is sum_j x_j W_hat[i][j] regrouped;
+ * the groups' terms are added in a fixed order, so repeated calls on the same
+ * inputs return the same y. The call is asynchronous: it returns once the kernels are enqueued on `stream` (host-side
  * argument checks only), so decode loops can issue it back to back. Workspace:
  * slim_dequant_gemv_workspace_bytes (0 when one launch covers every group of a
  * row, as for the usual layer shapes); ws NULL takes it from the library's
